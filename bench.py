@@ -1,0 +1,358 @@
+"""Benchmark of the AB-Attention hot path on B200.
+
+One step = one pass of the whole path (IBCS selector -> SIP sampler -> gather
+attention) over one batch of the synthetic Wan2.1-14B-720p-shaped workload
+(75,600 tokens, 40 heads, d = 128, 8 % block budget = 92 % skip).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl abatt|reference]
+
+Prints one JSON line (rank 0).  `value` is dense-equivalent TFLOPS
+(4 B H N^2 d per step / step time) summed over ranks; the roofline object
+covers the gather-attention kernel (executed 128x128 tiles, tensor bound).
+With N > 1 GPUs (torchrun), every rank runs its own batch element (heads are
+independent; no collective on the data path): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_20_b200 import synth  # noqa: E402
+
+METRIC = "attention ms & dense-equiv TFLOPS at 90% skip; % bf16 tensor peak (1 B200)"
+FALLBACK_PEAK_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="abatt", choices=["abatt", "reference"])
+    ap.add_argument("--workload", default="wan14b-720p", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--budget-bp", type=int, default=None, help="override (10000 = keep-all)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"bf16_tflops": FALLBACK_PEAK_TFLOPS, "bf16_tflops_sustained": 1400.0,
+                "hbm_gbs": 6650.0}, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_reference(args, w):
+    """The tier's reference arm: the float64 CPU oracle, as it stands, on a
+    bounded sample of query blocks per step."""
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cores = oracle.default_threads()
+    Q, K, V = synth.generate(w)
+    nrows = max(8, min(cores, 64))
+    stride = max(1, w.rows // nrows)
+    rows = np.arange(0, w.rows, stride)[:nrows]
+
+    def step():
+        oracle.forward(Q, K, V, w.shape, rows, w.clusters, w.iters, w.budget_bp, w.seed, Bk=w.Bk,
+                       nthreads=cores)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    full = dt * w.rows / len(rows)  # extrapolated to the whole workload
+    dense = 4.0 * w.B * w.H * w.N * w.N * w.d
+    value = dense / full / 1e12
+    sample = f"{len(rows)} of {w.rows} query blocks per step (every {stride}th), time x{w.rows / len(rows):.1f}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS (dense-equivalent)",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": full * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS (dense-equivalent)", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS (dense-equivalent)", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, Q, K, V, budget_s=15.0):
+    """The oracle on this host's cores, on a bounded sample of the workload."""
+    import oracle
+
+    cores = oracle.default_threads()
+    nrows = max(4, min(16 * cores, w.rows))
+    stride = max(1, w.rows // nrows)
+    rows = np.arange(0, w.rows, stride)[:nrows]
+    t0 = time.perf_counter()
+    oracle.forward(Q, K, V, w.shape, rows, w.clusters, w.iters, w.budget_bp, w.seed, Bk=w.Bk,
+                   nthreads=cores)
+    dt = time.perf_counter() - t0
+    full = dt * w.rows / len(rows)
+    dense = 4.0 * w.B * w.H * w.N * w.N * w.d
+    return {"value": dense / full / 1e12, "unit": "TFLOPS (dense-equivalent)", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{len(rows)} of {w.rows} query blocks (every {stride}th), {dt:.1f} s, "
+                      f"extrapolated x{w.rows / len(rows):.1f}"}
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    if args.budget_bp is not None:
+        w = w.with_(budget_bp=args.budget_bp)
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_attention_20_b200 import abatt
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    Qc, Kc, Vc = synth.generate(w)
+    Q, K, V = Qc.to(dev), Kc.to(dev), Vc.to(dev)
+    shape = w.shape
+    cfg = abatt.Config(kv_block=w.Bk, clusters=w.clusters, kmeans_iters=w.iters,
+                       budget_bp=w.budget_bp, seed=w.seed)
+    rows, nK = w.rows, w.nK
+    p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
+    counts = torch.empty(rows, dtype=torch.int32, device=dev)
+    idx = torch.empty((rows, nK), dtype=torch.int32, device=dev)
+    logw = torch.empty((rows, nK), dtype=torch.float32, device=dev)
+    O = torch.empty_like(Q)
+    ws_sel = torch.empty(abatt.workspace_size(abatt.CALL_SELECT, shape, cfg), dtype=torch.uint8,
+                         device=dev)
+    ws_small = torch.empty(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e: e[0].record(stream)
+        abatt.select(Q, K, cfg, p=p, workspace=ws_sel, stream=stream)
+        if e: e[1].record(stream)
+        abatt.sample(p, shape, cfg, out=(counts, idx, logw), workspace=ws_small, stream=stream)
+        if e: e[2].record(stream)
+        abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws_small, stream=stream)
+        if e: e[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for k in range(args.steps):
+            step(ev[k])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    sel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    smp_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    att_ms = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
+    att_mean = sum(e[2].elapsed_time(e[3]) for e in ev) / len(ev)
+    ms_step = total_ms / args.steps
+    status = abatt.read_status(ws_small) | abatt.read_status(ws_sel)
+
+    c = counts.cpu().numpy().astype(np.int64)
+    bpt = 128 // w.Bk
+    tiles = int(((c + bpt - 1) // bpt).sum())
+    exec_flop = tiles * 4.0 * 128 * 128 * w.d
+    # algorithmic work: valid query rows x valid drawn keys
+    nrows_q = np.minimum(128, w.N - (np.arange(rows) % w.nQ) * 128)
+    idx_h = idx.cpu().numpy()
+    keys = np.zeros(rows, dtype=np.int64)
+    last = w.nK - 1
+    tail = w.N - last * w.Bk
+    for r in range(rows):
+        L = c[r]
+        keys[r] = L * w.Bk - (w.Bk - tail if L and idx_h[r, :L][-1] == last else 0)
+    alg_flop = float((4.0 * w.d * nrows_q * keys).sum())
+    dense_flop = 4.0 * w.B * w.H * w.N * w.N * w.d
+    skip = 1.0 - float((nrows_q * keys).sum()) / (w.B * w.H * w.N * float(w.N))
+
+    pk, src = peaks()
+    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
+    achieved = exec_flop / (att_mean * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC,
+        "value": dense_flop * world / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOPS (dense-equivalent)",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters,
+                   "kmeans_iters": w.iters, "per_rank": "one batch element per GPU",
+                   "l2": "inputs (Q,K,V 2.3 GB) exceed the 126 MB L2; no flush"},
+        "stages_ms": {"select": sel_ms, "sample": smp_ms, "attention": att_ms},
+        "attention_ms": att_ms,
+        "selector_sampler_share": (sel_ms + smp_ms) / (sel_ms + smp_ms + att_ms),
+        "realized_skip": skip,
+        "executed_tflops_attention": achieved,
+        "algorithmic_tflops_attention": alg_flop / (att_mean * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "gather_attn_kernel", "peak_source": f"{src} bf16 sustained"},
+        "device_status": status,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world)
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, Qc, Kc, Vc)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):
+    """Same metric through the public call with host buffers: pinned H2D of
+    Q, K, V, abatt_forward, D2H of O, every step."""
+    import torch
+    import torch.distributed as dist
+
+    hq, hk, hv = (t.pin_memory() for t in (Qc, Kc, Vc))
+    ho = torch.empty_like(Qc).pin_memory()
+    Q, K, V = (torch.empty_like(t, device=dev) for t in (Qc, Kc, Vc))
+    O = torch.empty_like(Q)
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, w.shape, cfg), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        Q.copy_(hq, non_blocking=True)
+        K.copy_(hk, non_blocking=True)
+        V.copy_(hv, non_blocking=True)
+        abatt.forward(Q, K, V, cfg, out=O, workspace=ws, stream=stream)
+        ho.copy_(O, non_blocking=True)
+
+    steps = max(3, args.steps // 4)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    dense = 4.0 * w.B * w.H * w.N * w.N * w.d
+    nbytes = Qc.numel() * 2
+    return {"value": dense * world / (ms * 1e-3) / 1e12, "unit": "TFLOPS (dense-equivalent)",
+            "ms_per_step": ms, "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+            "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

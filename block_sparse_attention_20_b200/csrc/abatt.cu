@@ -1,0 +1,367 @@
+// abatt.cu -- host side of the C ABI declared in include/abatt.h: argument
+// validation, workspace layout, TMA descriptor encoding and the launch
+// sequence of each call.  No allocation, no synchronisation except in
+// abatt_read_status.
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "kernels.cuh"
+
+using namespace abatt;
+
+namespace {
+
+constexpr uint64_t kWaitNs = 500000000ull;  // bounded waits give up after ~0.5 s
+constexpr float kLog2eF = 1.4426950408889634f;
+
+struct Geom {
+    int B, H, N, d, Bq, Bk, C, I, nQ, nK, nT, ldr;
+    int64_t rows, heads, M;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
+    if (!s || !c) return ABATT_ERR_INVALID_ARG;
+    if (s->B <= 0 || s->H <= 0 || s->N <= 0 || s->d <= 0) return ABATT_ERR_INVALID_ARG;
+    if (c->budget_bp < 0 || !(c->scale > 0.0f) || !isfinite(c->scale)) return ABATT_ERR_INVALID_ARG;
+    if (s->d != 64 && s->d != 128) return ABATT_ERR_UNSUPPORTED;
+    if (c->q_block != 128) return ABATT_ERR_UNSUPPORTED;
+    if (c->kv_block != 16 && c->kv_block != 32 && c->kv_block != 64 && c->kv_block != 128)
+        return ABATT_ERR_UNSUPPORTED;
+    if (c->clusters < 1 || c->clusters > 16) return ABATT_ERR_UNSUPPORTED;
+    if (c->kmeans_iters < 0 || c->kmeans_iters > 64) return ABATT_ERR_UNSUPPORTED;
+    g->B = s->B; g->H = s->H; g->N = s->N; g->d = s->d;
+    g->Bq = c->q_block; g->Bk = c->kv_block; g->C = c->clusters; g->I = c->kmeans_iters;
+    g->nQ = (s->N + 127) / 128;
+    g->nK = (s->N + g->Bk - 1) / g->Bk;
+    g->nT = (s->N + 127) / 128;
+    g->ldr = g->nT * (128 / g->Bk);
+    g->heads = (int64_t)s->B * s->H;
+    g->rows = g->heads * g->nQ;
+    if (g->nK > 32767) return ABATT_ERR_UNSUPPORTED;
+    if (g->rows >= (int64_t(1) << 31) || g->heads > 65535) return ABATT_ERR_UNSUPPORTED;
+    if ((int64_t)s->N * s->d * g->heads >= (int64_t(1) << 40)) return ABATT_ERR_UNSUPPORTED;
+    g->M = ((int64_t)c->budget_bp * g->nK + 5000) / 10000;
+    return ABATT_OK;
+}
+
+// ---- workspace layout ----------------------------------------------------------
+struct Layout {
+    size_t hdr, cent_hi, cent_lo, weight, r, mref, mz;  // select
+    size_t p, counts, idx, logw;                          // forward
+    size_t total;
+};
+
+Layout layout(abatt_call call, const Geom &g) {
+    Layout L;
+    memset(&L, 0, sizeof L);
+    size_t off = 0;
+    L.hdr = off;
+    off += sizeof(WsHeader);
+    if (call == ABATT_CALL_SELECT || call == ABATT_CALL_FORWARD) {
+        const size_t crow = (size_t)g.rows * g.C;
+        L.cent_hi = off; off = align256(off + crow * g.d * 2);
+        L.cent_lo = off; off = align256(off + crow * g.d * 2);
+        L.weight = off;  off = align256(off + crow * 4);
+        L.r = off;       off = align256(off + crow * g.ldr * 4);
+        L.mref = off;    off = align256(off + crow * g.nT * 4);
+        L.mz = off;      off = align256(off + crow * 8);
+    }
+    if (call == ABATT_CALL_FORWARD) {
+        L.p = off;      off = align256(off + (size_t)g.rows * g.nK * 4);
+        L.counts = off; off = align256(off + (size_t)g.rows * 4);
+        L.idx = off;    off = align256(off + (size_t)g.rows * g.nK * 4);
+        L.logw = off;   off = align256(off + (size_t)g.rows * g.nK * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+// ---- per-device cache --------------------------------------------------------
+std::mutex g_mu;
+int g_sms[64];
+
+abatt_status device_sms(int *sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ABATT_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return ABATT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return ABATT_ERR_CUDA;
+        g_sms[dev] = n;
+    }
+    *sms = g_sms[dev];
+    return ABATT_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 map over [outer][rows][d] with a (64, box_rows, 1) box, 128-byte
+// swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t outer, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)outer};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+abatt_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ABATT_OK : ABATT_ERR_CUDA; }
+
+abatt_status check_ws(abatt_call call, const Geom &g, void *ws, size_t bytes) {
+    if (!ws) return ABATT_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ABATT_ERR_ALIGNMENT;
+    if (bytes < layout(call, g).total) return ABATT_ERR_WORKSPACE;
+    return ABATT_OK;
+}
+
+// ---- the three stages ------------------------------------------------------
+abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt_config *cfg,
+                        float *p, float *cent_out, int32_t *sizes_out, void *ws, const Layout &L,
+                        int sms, cudaStream_t st) {
+    KmeansArgs ka;
+    ka.Q = static_cast<const __nv_bfloat16 *>(Q);
+    ka.rows = g.rows; ka.nQ = g.nQ; ka.N = g.N; ka.D = g.d; ka.C = g.C; ka.iters = g.I;
+    ka.logit_mul = cfg->scale * kLog2eF;
+    ka.cent_hi = at<__nv_bfloat16>(ws, L.cent_hi);
+    ka.cent_lo = at<__nv_bfloat16>(ws, L.cent_lo);
+    ka.weight = at<float>(ws, L.weight);
+    ka.cent_out = cent_out;
+    ka.sizes_out = sizes_out;
+    cudaError_t e = launch_kmeans(ka, sms, st);
+    if (e != cudaSuccess) return ABATT_ERR_CUDA;
+
+    ScoreMaps sm;
+    const int64_t MC = (int64_t)g.nQ * g.C;
+    if (!make_map(&sm.a_hi, ka.cent_hi, g.d, MC, g.heads, 128) ||
+        !make_map(&sm.a_lo, ka.cent_lo, g.d, MC, g.heads, 128) ||
+        !make_map(&sm.k, K, g.d, g.N, g.heads, 128))
+        return ABATT_ERR_CUDA;
+    ScoreArgs sa;
+    sa.heads = (int)g.heads; sa.N = g.N; sa.D = g.d; sa.Bk = g.Bk; sa.MC = (int)MC;
+    sa.nT = g.nT; sa.ldr = g.ldr; sa.use_lo = 1;
+    sa.r = at<float>(ws, L.r);
+    sa.mref = at<float>(ws, L.mref);
+    sa.mz = at<float2>(ws, L.mz);
+    sa.hdr = at<WsHeader>(ws, L.hdr);
+    sa.wait_ns = kWaitNs;
+    e = launch_score(sa, sm, sms, st);
+    if (e != cudaSuccess) return ABATT_ERR_CUDA;
+
+    CombineArgs ca;
+    ca.rows = g.rows; ca.C = g.C; ca.nK = g.nK; ca.nT = g.nT; ca.ldr = g.ldr; ca.Bk = g.Bk;
+    ca.r = sa.r; ca.mref = sa.mref; ca.weight = ka.weight; ca.mz = sa.mz; ca.p = p;
+    return cuda_status(launch_combine(ca, sms, st));
+}
+
+abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, int32_t *counts,
+                        int32_t *idx, float *logw, int capacity, WsHeader *hdr, int sms,
+                        cudaStream_t st) {
+    SampleArgs a;
+    a.p = p; a.rows = g.rows; a.nK = g.nK; a.nK_pad = (g.nK + 3) & ~3; a.nQ = g.nQ; a.H = g.H;
+    a.M = g.M;
+    a.key0 = (uint32_t)(cfg->seed & 0xffffffffu);
+    a.key1 = (uint32_t)(cfg->seed >> 32);
+    a.capacity = capacity; a.counts = counts; a.idx = idx; a.logw = logw;
+    a.status = &hdr->status;
+    return cuda_status(launch_sample(a, sms, st));
+}
+
+abatt_status run_attention(const void *Q, const void *K, const void *V, const Geom &g,
+                           const abatt_config *cfg, const int32_t *counts, const int32_t *idx,
+                           const float *logw, int capacity, void *O, float *lse, WsHeader *hdr,
+                           int sms, cudaStream_t st) {
+    AttnMaps m;
+    if (!make_map(&m.q, Q, g.d, g.N, g.heads, 128) || !make_map(&m.k, K, g.d, g.N, g.heads, g.Bk) ||
+        !make_map(&m.v, V, g.d, g.N, g.heads, g.Bk))
+        return ABATT_ERR_CUDA;
+    AttnArgs a;
+    a.rows = g.rows; a.nQ = g.nQ; a.N = g.N; a.D = g.d; a.Bk = g.Bk; a.nK = g.nK;
+    a.capacity = capacity;
+    a.scale_log2 = cfg->scale * kLog2eF;
+    a.counts = counts; a.idx = idx; a.logw = logw;
+    a.O = static_cast<__nv_bfloat16 *>(O);
+    a.lse = lse;
+    a.hdr = hdr;
+    a.wait_ns = kWaitNs;
+    return cuda_status(launch_attention(a, m, sms, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *abatt_version(void) { return "0.1.0"; }
+
+const char *abatt_status_string(abatt_status s) {
+    switch (s) {
+        case ABATT_OK: return "ok";
+        case ABATT_ERR_INVALID_ARG: return "invalid argument";
+        case ABATT_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+        case ABATT_ERR_ALIGNMENT: return "misaligned pointer";
+        case ABATT_ERR_WORKSPACE: return "workspace missing or too small";
+        case ABATT_ERR_CUDA: return "CUDA runtime error";
+        case ABATT_ERR_CAPACITY: return "a row drew more blocks than the list capacity";
+        case ABATT_ERR_TIMEOUT: return "a bounded device wait ran out";
+        case ABATT_ERR_DEVICE: return "device status word reports an error";
+    }
+    return "unknown status";
+}
+
+abatt_status abatt_workspace_size(abatt_call call, const abatt_shape *shape,
+                                  const abatt_config *cfg, size_t *bytes) {
+    if (!bytes) return ABATT_ERR_INVALID_ARG;
+    if (call < ABATT_CALL_SELECT || call > ABATT_CALL_FORWARD) return ABATT_ERR_INVALID_ARG;
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    *bytes = layout(call, g).total;
+    return ABATT_OK;
+}
+
+abatt_status abatt_select(const void *Q, const void *K, const abatt_shape *shape,
+                          const abatt_config *cfg, float *p, float *centroids,
+                          int32_t *cluster_sizes, void *workspace, size_t workspace_bytes,
+                          void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!Q || !K || !p) return ABATT_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(p)) return ABATT_ERR_ALIGNMENT;
+    if ((s = check_ws(ABATT_CALL_SELECT, g, workspace, workspace_bytes)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Layout L = layout(ABATT_CALL_SELECT, g);
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
+    return run_select(Q, K, g, cfg, p, centroids, cluster_sizes, workspace, L, sms, st);
+}
+
+abatt_status abatt_sample(const float *p, const abatt_shape *shape, const abatt_config *cfg,
+                          int32_t *counts, int32_t *idx, float *logw, int capacity,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!p || !counts || !idx || !logw || capacity < 1) return ABATT_ERR_INVALID_ARG;
+    if ((s = check_ws(ABATT_CALL_SAMPLE, g, workspace, workspace_bytes)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
+    return run_sample(p, g, cfg, counts, idx, logw, capacity, static_cast<WsHeader *>(workspace),
+                      sms, st);
+}
+
+abatt_status abatt_attention(const void *Q, const void *K, const void *V,
+                             const abatt_shape *shape, const abatt_config *cfg,
+                             const int32_t *counts, const int32_t *idx, const float *logw,
+                             int capacity, void *O, float *lse, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!Q || !K || !V || !O || !counts || !idx || !logw || capacity < 1)
+        return ABATT_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return ABATT_ERR_ALIGNMENT;
+    if ((s = check_ws(ABATT_CALL_ATTENTION, g, workspace, workspace_bytes)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
+    return run_attention(Q, K, V, g, cfg, counts, idx, logw, capacity, O, lse,
+                         static_cast<WsHeader *>(workspace), sms, st);
+}
+
+abatt_status abatt_forward(const void *Q, const void *K, const void *V,
+                           const abatt_shape *shape, const abatt_config *cfg, void *O,
+                           float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!Q || !K || !V || !O) return ABATT_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return ABATT_ERR_ALIGNMENT;
+    if ((s = check_ws(ABATT_CALL_FORWARD, g, workspace, workspace_bytes)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Layout L = layout(ABATT_CALL_FORWARD, g);
+    WsHeader *hdr = at<WsHeader>(workspace, L.hdr);
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
+    float *p = at<float>(workspace, L.p);
+    int32_t *counts = at<int32_t>(workspace, L.counts);
+    int32_t *idx = at<int32_t>(workspace, L.idx);
+    float *logw = at<float>(workspace, L.logw);
+    if ((s = run_select(Q, K, g, cfg, p, nullptr, nullptr, workspace, L, sms, st)) != ABATT_OK)
+        return s;
+    if ((s = run_sample(p, g, cfg, counts, idx, logw, g.nK, hdr, sms, st)) != ABATT_OK) return s;
+    return run_attention(Q, K, V, g, cfg, counts, idx, logw, g.nK, O, lse, hdr, sms, st);
+}
+
+abatt_status abatt_forward_intermediates(void *workspace, const abatt_shape *shape,
+                                         const abatt_config *cfg, float **p, int32_t **counts,
+                                         int32_t **idx, float **logw) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!workspace) return ABATT_ERR_WORKSPACE;
+    const Layout L = layout(ABATT_CALL_FORWARD, g);
+    if (p) *p = at<float>(workspace, L.p);
+    if (counts) *counts = at<int32_t>(workspace, L.counts);
+    if (idx) *idx = at<int32_t>(workspace, L.idx);
+    if (logw) *logw = at<float>(workspace, L.logw);
+    return ABATT_OK;
+}
+
+abatt_status abatt_read_status(const void *workspace, uint32_t *flags, void *stream) {
+    if (!workspace || !flags) return ABATT_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return ABATT_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return ABATT_ERR_CUDA;
+    *flags = v;
+    return v ? ABATT_ERR_DEVICE : ABATT_OK;
+}
+
+abatt_status abatt_clear_status(void *workspace, void *stream) {
+    if (!workspace) return ABATT_ERR_INVALID_ARG;
+    return cuda_status(
+        cudaMemsetAsync(workspace, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// kernels.cuh -- argument blocks and launchers of the abatt kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace abatt {
+
+// ---- IBCS part 1: per-query-block k-means ---------------------------------
+struct KmeansArgs {
+    const __nv_bfloat16 *Q;  // [B*H][N][D]
+    int64_t rows;            // B*H*nQ
+    int nQ, N, D, C, iters;
+    float logit_mul;         // scale * log2(e), folded into the GEMM operand
+    __nv_bfloat16 *cent_hi;  // [rows*C][D]
+    __nv_bfloat16 *cent_lo;  // [rows*C][D]
+    float *weight;           // [rows][C]  n_j / n
+    float *cent_out;         // optional [rows][C][D]
+    int32_t *sizes_out;      // optional [rows][C]
+};
+size_t kmeans_smem_bytes(int D);
+cudaError_t launch_kmeans(const KmeansArgs &a, int num_sms, cudaStream_t stream);
+
+// ---- IBCS part 2: centroid . key softmax mass per key block -----------------
+// For every centroid row (head hd, local row m < MC = nQ*C) and every 128-key
+// tile T: base-2 logits x = c'.k (c' pre-scaled), running max and sum, and
+// per key block b of the tile the partial mass r = sum_{t in b} 2^(x - mref_T)
+// where mref_T is the row's running maximum after tile T.
+struct ScoreArgs {
+    int heads;     // B*H
+    int N, D, Bk;
+    int MC;        // centroid rows per head (nQ*C)
+    int nT;        // key tiles per head, ceil(N/128)
+    int ldr;       // row stride of r in floats (nT * 128/Bk)
+    int use_lo;    // add the lo half of the split centroids (fp32-accurate logits)
+    float *r;      // [heads*MC][ldr]
+    float *mref;   // [heads*MC][nT]
+    float2 *mz;    // [heads*MC] (final max, sum) in base 2
+    WsHeader *hdr;
+    uint64_t wait_ns;
+};
+struct ScoreMaps {
+    CUtensorMap a_hi, a_lo, k;
+};
+cudaError_t launch_score(const ScoreArgs &a, const ScoreMaps &maps, int num_sms,
+                         cudaStream_t stream);
+
+// Combine the C centroids of each query block into p (see score.cu).
+struct CombineArgs {
+    int64_t rows;  // query blocks
+    int C, nK, nT, ldr, Bk;
+    const float *r, *mref, *weight;
+    const float2 *mz;
+    float *p;      // [rows][nK]
+};
+cudaError_t launch_combine(const CombineArgs &a, int num_sms, cudaStream_t stream);
+
+// ---- SIP sampler --------------------------------------------------------
+struct SampleArgs {
+    const float *p;  // [rows][nK]
+    int64_t rows;
+    int nK, nK_pad, nQ, H;
+    int64_t M;
+    uint32_t key0, key1;
+    int capacity;
+    int32_t *counts, *idx;
+    float *logw;
+    uint32_t *status;
+};
+size_t sample_smem_bytes(int nK);
+cudaError_t launch_sample(const SampleArgs &a, int num_sms, cudaStream_t stream);
+
+// ---- gather attention -----------------------------------------------------
+struct AttnArgs {
+    int64_t rows;  // query blocks
+    int nQ, N, D, Bk, nK;
+    int capacity;
+    float scale_log2;  // scale * log2(e)
+    const int32_t *counts, *idx;
+    const float *logw;
+    __nv_bfloat16 *O;  // [B*H][N][D]
+    float *lse;        // optional [B*H][N]
+    WsHeader *hdr;
+    uint64_t wait_ns;
+};
+struct AttnMaps {
+    CUtensorMap q, k, v;
+};
+cudaError_t launch_attention(const AttnArgs &a, const AttnMaps &maps, int num_sms,
+                             cudaStream_t stream);
+
+}  // namespace abatt

@@ -1,0 +1,171 @@
+/*
+ * abatt.h -- C ABI of the AB-Attention hot path on B200 (sm_100a).
+ *
+ * Method: "Accurate Block Attention (AB-Attention)", abstract.  Dynamic
+ * block-sparse attention for video diffusion transformers in three stages:
+ *   IBCS  the queries of each query block are clustered on their own (no
+ *         token reordering) and the centroids estimate how much attention
+ *         mass every key/value block receives;
+ *   SIP   key/value blocks are drawn with probability proportional to those
+ *         estimates and re-weighted by 1/(inclusion probability), so that one
+ *         pass estimates dense attention instead of truncating it;
+ *   gather kernel: the drawn key/value blocks (much smaller than a tile) are
+ *         packed into full tensor-core tiles.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device.
+ *     The caller owns every buffer; the library never allocates or frees
+ *     memory and keeps no state between calls other than cached kernel
+ *     attributes.
+ *   - Q, K, V, O: bf16, contiguous [B][H][N][d], 16-byte aligned base.
+ *   - A "row" is one query block (beta, h, i), linear id
+ *     ((beta*H)+h)*nQ + i, with nQ = ceil(N/q_block), nK = ceil(N/kv_block).
+ *     The last query block and the last key block may be partial; missing
+ *     rows/keys do not exist (masked from every softmax, never stored).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream.
+ *   - Errors found on the host return immediately, before any launch.
+ *     Errors found on the device (list overflow, a bounded wait that ran
+ *     out) are OR-ed as ABATT_DEVFLAG_* bits into the 32-bit status word at
+ *     the start of the call's workspace; read it with abatt_read_status.
+ *     Nothing traps or spins without bound on the device.
+ *   - Limits: d in {64, 128}; q_block == 128; kv_block in {16, 32, 64, 128};
+ *     1 <= clusters <= 16; 0 <= kmeans_iters <= 64; nK <= 32767;
+ *     B*H*nQ < 2^31.
+ */
+#ifndef ABATT_H
+#define ABATT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum abatt_status {
+    ABATT_OK = 0,
+    ABATT_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad budget */
+    ABATT_ERR_UNSUPPORTED = 2, /* a limit above is exceeded */
+    ABATT_ERR_ALIGNMENT = 3,   /* a tensor base is not 16-byte aligned */
+    ABATT_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+    ABATT_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    ABATT_ERR_CAPACITY = 6,    /* (device) a row drew more blocks than capacity */
+    ABATT_ERR_TIMEOUT = 7,     /* (device) a bounded wait ran out */
+    ABATT_ERR_DEVICE = 8       /* device status word holds an error */
+} abatt_status;
+
+/* Bits of the device status word. */
+#define ABATT_DEVFLAG_CAPACITY 0x1u
+#define ABATT_DEVFLAG_TIMEOUT 0x2u
+#define ABATT_DEVFLAG_BADLIST 0x4u /* a block index outside [0, nK) was skipped */
+
+typedef struct abatt_shape {
+    int B; /* batch */
+    int H; /* heads */
+    int N; /* tokens (the flattened latent video grid, raster order) */
+    int d; /* head dimension */
+} abatt_shape;
+
+typedef struct abatt_config {
+    int q_block;        /* Bq: queries per query block (128) */
+    int kv_block;       /* Bk: keys per key/value block (16 by default) */
+    int clusters;       /* C: k-means clusters per query block */
+    int kmeans_iters;   /* I: Lloyd rounds (assign + update) */
+    int budget_bp;      /* expected drawn blocks, basis points of nK:
+                           M = floor((budget_bp*nK + 5000)/10000); M >= nK
+                           keeps every block with weight 1 */
+    float scale;        /* softmax scale s (1/sqrt(d) for plain attention) */
+    uint64_t seed;      /* Philox key for the draws */
+} abatt_config;
+
+/* Which call a workspace is for. */
+typedef enum abatt_call {
+    ABATT_CALL_SELECT = 0,
+    ABATT_CALL_SAMPLE = 1,
+    ABATT_CALL_ATTENTION = 2,
+    ABATT_CALL_FORWARD = 3
+} abatt_call;
+
+/* Bytes of device workspace `call` needs for this shape/config (256-byte
+ * aligned base).  `capacity` is the list capacity used by ATTENTION
+ * (ignored otherwise).  Host-only, no CUDA call. */
+abatt_status abatt_workspace_size(abatt_call call, const abatt_shape *shape,
+                                  const abatt_config *cfg, size_t *bytes);
+
+/* IBCS (abstract, selector sentence): for every query block, Lloyd k-means of
+ * its valid queries (C_eff = min(C, n) clusters seeded at rows
+ * floor(j*n/C_eff), ties to the lower index, empty clusters keep their
+ * centroid), then each centroid's softmax (scale s) mass over all keys,
+ * summed per key block and weighted by the cluster's share n_j/n:
+ *   p[row][b] = sum_j (n_j/n) * sum_{t in block b} softmax_t(s c_j . k_t).
+ * Output p: fp32 [B*H*nQ][nK], each row sums to 1.
+ * Optional outputs (NULL to skip): centroids fp32 [B*H*nQ][C][d] and
+ * cluster sizes int32 [B*H*nQ][C] (0 for unused clusters). */
+abatt_status abatt_select(const void *Q, const void *K, const abatt_shape *shape,
+                          const abatt_config *cfg, float *p, float *centroids,
+                          int32_t *cluster_sizes, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* SIP (abstract, sampling sentence): Poisson draw of key blocks per row with
+ * inclusion probabilities pi_b = min(1, c p_b), sum_b pi_b = M, solved
+ * exactly in 48-bit fixed point (P_b = round-half-even(p_b 2^48), p clamped
+ * to [0,1], NaN read as 0; water-filling of the saturated set).  Draw U_b is
+ * word (b mod 4) of Philox4x32-10 at counter (b/4, i, h, beta), key
+ * (seed lo, seed hi); block b is taken iff saturated or U_b/2^32 < pi_b
+ * (exact integer test).
+ * Outputs: counts int32 [rows]; idx int32 [rows][capacity] in ascending
+ * order; logw fp32 [rows][capacity] = -ln(pi_b) (0 when pi_b = 1).  A row
+ * that draws more than `capacity` blocks keeps the first `capacity` and sets
+ * ABATT_DEVFLAG_CAPACITY.  Results are bit-identical for any launch
+ * configuration, stream or device. */
+abatt_status abatt_sample(const float *p, const abatt_shape *shape, const abatt_config *cfg,
+                          int32_t *counts, int32_t *idx, float *logw, int capacity,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Gather attention (abstract, kernel sentence): for every query block, exact
+ * softmax attention over the keys of its listed blocks only, each logit of
+ * block b shifted by logw_b:
+ *   O[q] = sum_t e^{l_t} v_t / sum_t e^{l_t},  l_t = s q.k_t + logw_{b(t)}.
+ * Blocks are gathered from K/V into 128-key tensor-core tiles.  An empty
+ * list gives O = 0 (and lse = -inf).  lse (optional, NULL to skip): fp32
+ * [B][H][N], natural-log sum of exponentials per query.  Indices outside
+ * [0, nK) are skipped and flagged ABATT_DEVFLAG_BADLIST. */
+abatt_status abatt_attention(const void *Q, const void *K, const void *V,
+                             const abatt_shape *shape, const abatt_config *cfg,
+                             const int32_t *counts, const int32_t *idx, const float *logw,
+                             int capacity, void *O, float *lse, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/* The whole path: select -> sample -> attention, on one stream, with p and the
+ * lists kept in the workspace (capacity nK, so no row can overflow). */
+abatt_status abatt_forward(const void *Q, const void *K, const void *V,
+                           const abatt_shape *shape, const abatt_config *cfg, void *O,
+                           float *lse, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Pointers into a FORWARD workspace (valid after abatt_forward completes):
+ * p fp32 [rows][nK], counts int32 [rows], idx int32 [rows][nK],
+ * logw fp32 [rows][nK].  Any output pointer may be NULL. */
+abatt_status abatt_forward_intermediates(void *workspace, const abatt_shape *shape,
+                                         const abatt_config *cfg, float **p, int32_t **counts,
+                                         int32_t **idx, float **logw);
+
+/* Synchronously copy the device status word at the start of `workspace` to
+ * *flags (ABATT_DEVFLAG_* bits) after `stream` drains.  Returns
+ * ABATT_ERR_DEVICE if any bit is set, ABATT_OK otherwise. */
+abatt_status abatt_read_status(const void *workspace, uint32_t *flags, void *stream);
+
+/* Zero the device status word (asynchronous on `stream`). */
+abatt_status abatt_clear_status(void *workspace, void *stream);
+
+/* Static description of a status code. */
+const char *abatt_status_string(abatt_status s);
+
+/* Library version "major.minor.patch". */
+const char *abatt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ABATT_H */

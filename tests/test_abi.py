@@ -1,0 +1,115 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point declared in include/abatt.h, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_20_b200 import abatt, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return abatt.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "abatt.h")).read()
+    return sorted(set(re.findall(r"^\S.*?\b(abatt_\w+)\(", src, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 10
+    assert sorted(abatt.EXPORTS) == names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert re.match(r"\d+\.\d+\.\d+$", abatt.version())
+    for code in range(9):
+        assert abatt.status_string(code) not in ("", "unknown status")
+    assert abatt.status_string(99) == "unknown status"
+
+
+def _ws(shape, cfg, call=abatt.CALL_FORWARD):
+    return abatt.workspace_size(call, shape, cfg)
+
+
+def test_workspace_sizes():
+    cfg = abatt.Config(clusters=8, budget_bp=800)
+    B, H, N, d = 1, 40, 75600, 128
+    fwd = _ws((B, H, N, d), cfg)
+    sel = _ws((B, H, N, d), cfg, abatt.CALL_SELECT)
+    assert _ws((B, H, N, d), cfg, abatt.CALL_SAMPLE) == 256
+    assert _ws((B, H, N, d), cfg, abatt.CALL_ATTENTION) == 256
+    rows, nK = 40 * 591, 4725
+    # forward holds the selector's scratch plus p and capacity-nK lists
+    assert fwd >= sel + rows * nK * 12 + rows * 4
+    assert fwd < 8 * 2**30
+
+
+@pytest.mark.parametrize("shape,kw,code", [
+    ((1, 1, 100, 96), {}, 2),            # d not in {64, 128}
+    ((1, 1, 100, 64), {"q_block": 64}, 2),
+    ((1, 1, 100, 64), {"kv_block": 8}, 2),
+    ((1, 1, 100, 64), {"clusters": 17}, 2),
+    ((1, 1, 100, 64), {"clusters": 0}, 2),
+    ((1, 1, 100, 64), {"kmeans_iters": 65}, 2),
+    ((1, 1, 16 * 32768, 64), {}, 2),      # nK > 32767
+    ((0, 1, 100, 64), {}, 1),
+    ((1, 1, 0, 64), {}, 1),
+    ((1, 1, 100, 64), {"budget_bp": -1}, 1),
+    ((1, 1, 100, 64), {"scale": 0.0}, 1),
+    ((1, 1, 100, 64), {"scale": float("nan")}, 1),
+])
+def test_validation(shape, kw, code):
+    with pytest.raises(abatt.AbattError) as e:
+        _ws(shape, abatt.Config(**kw))
+    assert e.value.code == code
+
+
+def test_host_side_rejections_before_any_device_call(L):
+    sh = abatt._Shape(1, 2, 256, 64)
+    cfg = abatt.Config()._c(64)
+    P = ctypes.c_void_p
+    # null tensors
+    assert L.abatt_select(None, None, ctypes.byref(sh), ctypes.byref(cfg), None, None, None,
+                          None, 0, None) == 1
+    assert L.abatt_attention(None, None, None, ctypes.byref(sh), ctypes.byref(cfg), None, None,
+                             None, 16, None, None, None, 0, None) == 1
+    assert L.abatt_forward(None, None, None, ctypes.byref(sh), ctypes.byref(cfg), None, None,
+                           None, 0, None) == 1
+    # misaligned tensor pointers (never dereferenced)
+    odd = P(0x1001)
+    assert L.abatt_forward(odd, odd, odd, ctypes.byref(sh), ctypes.byref(cfg), odd, None,
+                           P(0x100000), 1 << 30, None) == 3
+    # missing / small / misaligned workspace
+    ok = P(0x100000)
+    assert L.abatt_forward(ok, ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, None, None, 0,
+                           None) == 4
+    assert L.abatt_forward(ok, ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, None, ok, 255,
+                           None) == 4
+    assert L.abatt_forward(ok, ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, None,
+                           P(0x100010), 1 << 30, None) == 3
+    # sample: capacity must be positive
+    assert L.abatt_sample(ok, ctypes.byref(sh), ctypes.byref(cfg), ok, ok, ok, 0, ok, 256,
+                          None) == 1
+    # null shape / config
+    assert L.abatt_forward(ok, ok, ok, None, ctypes.byref(cfg), ok, None, ok, 1 << 30, None) == 1
+    size = ctypes.c_size_t()
+    assert L.abatt_workspace_size(7, ctypes.byref(sh), ctypes.byref(cfg), ctypes.byref(size)) == 1
+    assert L.abatt_read_status(None, None, None) == 1
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(abatt, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(abatt, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        abatt.lib()

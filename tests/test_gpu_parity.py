@@ -1,0 +1,319 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Matching rules:
+  - sampler fed the oracle's fp32 probabilities: counts, indices and
+    log-weights bit-exact (a log-weight may differ by one ulp only where the
+    oracle flags its fp32 rounding as too close to call);
+  - gather attention fed the same lists: relative L2 error <= 5e-3 and max
+    abs error <= 2e-2 against the oracle (bf16 inputs, fp32 accumulation);
+  - selector: probabilities close to the oracle's, and end-to-end sampled
+    block agreement >= 99.9 % with the same seed;
+  - at the benchmark's full size (75,600 tokens, 40 heads): the same checks on
+    sampled rows the oracle computes one by one, plus properties that hold at
+    any size (p sums to one, list invariants, the realised budget).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_20_b200 import abatt, synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 5e-3
+MAX_ABS = 2e-2
+AGREE = 0.999
+
+
+def cfg_of(w, **kw):
+    base = dict(kv_block=w.Bk, clusters=w.clusters, kmeans_iters=w.iters, budget_bp=w.budget_bp,
+                seed=w.seed)
+    base.update(kw)
+    return abatt.Config(**base)
+
+
+def _rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def _sets(counts, idx):
+    return [set(idx[r, :counts[r]].tolist()) for r in range(len(counts))]
+
+
+def agreement(c_gpu, i_gpu, c_orc, i_orc):
+    sg, so = _sets(c_gpu, i_gpu), _sets(c_orc, i_orc)
+    diff = sum(len(a ^ b) for a, b in zip(sg, so))
+    tot = sum(len(b) for b in so)
+    return 1.0 - diff / max(tot, 1)
+
+
+def _check_lists_exact(counts, idx, logw, oc, oi, ol, oamb):
+    assert np.array_equal(counts, oc)
+    for r in range(len(counts)):
+        L = counts[r]
+        assert np.array_equal(idx[r, :L], oi[r, :L]), r
+        a, b = logw[r, :L], ol[r, :L]
+        same = a.view(np.uint32) == b.view(np.uint32)
+        if not same.all():
+            bad = ~same
+            assert oamb[r, :L][bad].all(), (r, a[bad], b[bad])
+            assert np.all(np.abs(a[bad].view(np.int32) - b[bad].view(np.int32)) == 1)
+
+
+def _rows_of(shape, Bq=128):
+    B, H, N, d = shape
+    return np.arange(B * H * (-(-N // Bq)))
+
+
+# ---------------------------------------------------------------------------- sampler
+
+@pytest.mark.parametrize("nK,Bk,bp,conc", [(256, 16, 1000, 0.3), (4725, 16, 800, 0.05),
+                                           (7425, 16, 1100, 0.2), (63, 16, 2500, 1.0),
+                                           (8192, 16, 500, 0.1), (1, 128, 1000, 1.0),
+                                           (3, 64, 9000, 0.5), (64, 32, 10000, 0.3),
+                                           (100, 16, 0, 0.3)])
+def test_sample_bit_exact(nK, Bk, bp, conc):
+    N = nK * Bk - (Bk // 2 if nK > 1 else 0)
+    shape = (1, 2, N, 64)
+    rows = _rows_of(shape)
+    p = synth.random_probs(len(rows), nK, 1000 + nK, conc)
+    # special rows: all zero, one-hot, NaN / negative / > 1 entries, uniform
+    p[0] = 0
+    if len(rows) > 3:
+        p[1] = 0; p[1, nK // 2] = 1
+        p[2, 0] = np.nan; p[2, -1] = -1; p[2, nK // 3] = 3.0
+        p[3] = 1.0 / nK
+    cfg = abatt.Config(kv_block=Bk, budget_bp=bp, seed=0xDEADBEEF12345678)
+    c, i, lw, ws = abatt.sample(torch.from_numpy(p).cuda(), shape, cfg)
+    assert abatt.read_status(ws) == 0
+    oc, oi, ol, oamb, of = oracle.sample(p, shape, rows, bp, cfg.seed, Bk=Bk)
+    _check_lists_exact(c.cpu().numpy(), i.cpu().numpy(), lw.cpu().numpy(), oc, oi, ol, oamb)
+
+
+def test_sample_capacity_overflow_flags_and_truncates():
+    nK, Bk = 512, 16
+    shape = (1, 1, nK * Bk, 64)
+    rows = _rows_of(shape)
+    p = synth.random_probs(len(rows), nK, 7, 0.5)
+    cfg = abatt.Config(kv_block=Bk, budget_bp=2000, seed=3)
+    oc, oi, ol, oamb, _ = oracle.sample(p, shape, rows, 2000, 3, Bk=Bk)
+    cap = int(oc.min()) - 2
+    c, i, lw, ws = abatt.sample(torch.from_numpy(p).cuda(), shape, cfg, capacity=cap)
+    assert abatt.read_status(ws) & abatt.DEVFLAG_CAPACITY
+    c, i = c.cpu().numpy(), i.cpu().numpy()
+    assert np.all(c == cap)
+    for r in range(len(rows)):
+        assert np.array_equal(i[r], oi[r, :cap])
+
+
+def test_sample_repeatable_on_other_stream():
+    nK, Bk = 4725, 16
+    shape = (1, 3, nK * Bk, 128)
+    p = torch.from_numpy(synth.random_probs(len(_rows_of(shape)), nK, 9, 0.1)).cuda()
+    cfg = abatt.Config(kv_block=Bk, budget_bp=800, seed=11)
+    a = abatt.sample(p, shape, cfg)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = abatt.sample(p, shape, cfg, stream=s)
+    s.synchronize()
+    for x, y in zip(a[:3], b[:3]):
+        assert torch.equal(x, y)
+
+
+# -------------------------------------------------------------------------- attention
+
+def _random_lists(shape, Bk, bp, seed, conc=0.3):
+    B, H, N, d = shape
+    nK = -(-N // Bk)
+    rows = _rows_of(shape)
+    p = synth.random_probs(len(rows), nK, seed, conc)
+    c, i, lw, amb, _ = oracle.sample(p, shape, rows, bp, seed, Bk=Bk)
+    return rows, c, i, lw
+
+
+def _attn_check(Q, K, V, shape, Bk, rows, c, i, lw, scale=None):
+    cfg = abatt.Config(kv_block=Bk, scale=scale)
+    O, lse = abatt.attention(Q.cuda(), K.cuda(), V.cuda(), torch.from_numpy(c).cuda(),
+                             torch.from_numpy(i).cuda(), torch.from_numpy(lw).cuda(), cfg,
+                             want_lse=True)
+    O = O.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    ref, ref_lse = oracle.ht_attention(Q, K, V, shape, rows, c, i, lw, Bk=Bk, scale=scale)
+    B, H, N, d = shape
+    nQ = -(-N // 128)
+    got = np.zeros_like(ref)
+    got_lse = np.full_like(ref_lse, -np.inf)
+    for r in rows:
+        bh, q = divmod(int(r), nQ)
+        b, h = divmod(bh, H)
+        n = min(128, N - q * 128)
+        got[r, :n] = O[b, h, q * 128:q * 128 + n]
+        got_lse[r, :n] = lse[b, h, q * 128:q * 128 + n]
+    assert _rel_l2(got, ref) <= REL_L2
+    assert np.max(np.abs(got - ref)) <= MAX_ABS
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(fin, np.isfinite(got_lse))
+    assert np.max(np.abs(got_lse[fin] - ref_lse[fin])) <= 1e-2
+    return got, ref
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Bk", [16, 32, 64, 128])
+def test_attention_ragged_shapes(d, Bk):
+    shape = (2, 2, 1000, d)  # nQ = 8 (last block 104 rows), partial last key block
+    Q, K, V = (synth.random_bf16(shape, s) for s in (1, 2, 3))
+    rows, c, i, lw = _random_lists(shape, Bk, 2500, 17 + Bk)
+    _attn_check(Q, K, V, shape, Bk, rows, c, i, lw)
+
+
+def test_attention_tiny_oracle_lists():
+    w = synth.TINY
+    Q, K, V = synth.generate(w)
+    rows = _rows_of(w.shape)
+    _, p32 = oracle.block_probs(Q, K, w.shape, rows, w.clusters, w.iters, Bk=w.Bk)
+    c, i, lw, amb, _ = oracle.sample(p32, w.shape, rows, w.budget_bp, w.seed, Bk=w.Bk)
+    _attn_check(Q, K, V, w.shape, w.Bk, rows, c, i, lw)
+
+
+def test_attention_keep_all_is_dense():
+    shape = (1, 2, 700, 128)
+    Q, K, V = (synth.random_bf16(shape, s, 1.5) for s in (4, 5, 6))
+    Bk = 16
+    rows = _rows_of(shape)
+    nK = -(-700 // Bk)
+    c = np.full(len(rows), nK, np.int32)
+    i = np.tile(np.arange(nK, dtype=np.int32), (len(rows), 1))
+    lw = np.zeros((len(rows), nK), np.float32)
+    got, _ = _attn_check(Q, K, V, shape, Bk, rows, c, i, lw)
+    dense = oracle.dense_attention(Q, K, V, shape, rows)
+    assert _rel_l2(got, dense) <= REL_L2
+
+
+def test_attention_large_logweights_and_scale():
+    shape = (1, 1, 2048, 128)
+    Q, K, V = (synth.random_bf16(shape, s, 2.0) for s in (7, 8, 9))
+    rows, c, i, lw = _random_lists(shape, 16, 300, 23, conc=0.02)  # tiny pi -> large weights
+    assert lw.max() > 5
+    _attn_check(Q, K, V, shape, 16, rows, c, i, lw, scale=0.2)
+
+
+def test_attention_empty_rows_and_bad_index():
+    shape = (1, 2, 512, 64)
+    Q, K, V = (synth.random_bf16(shape, s) for s in (10, 11, 12))
+    rows, c, i, lw = _random_lists(shape, 16, 2000, 31)
+    c[0] = 0
+    c[3] = 0
+    _attn_check(Q, K, V, shape, 16, rows, c, i, lw)
+    # an out-of-range index is skipped and flagged
+    i2 = i.copy()
+    i2[1, 0] = 10**6
+    cfg = abatt.Config(kv_block=16)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    O = abatt.attention(Q.cuda(), K.cuda(), V.cuda(), torch.from_numpy(c).cuda(),
+                        torch.from_numpy(i2).cuda(), torch.from_numpy(lw).cuda(), cfg,
+                        workspace=ws)
+    assert abatt.read_status(ws) & abatt.DEVFLAG_BADLIST
+    keep = np.ones(c[1], bool)
+    keep[0] = False
+    i3 = i.copy()
+    i3[1, :c[1] - 1] = i[1, :c[1]][keep]
+    lw3 = lw.copy()
+    lw3[1, :c[1] - 1] = lw[1, :c[1]][keep]
+    c3 = c.copy()
+    c3[1] -= 1
+    ref, _ = oracle.ht_attention(Q, K, V, shape, rows, c3, i3, lw3, Bk=16)
+    got = O.float().cpu().numpy()[0, 0, 128:256]
+    assert _rel_l2(got, ref[1]) <= REL_L2
+
+
+# --------------------------------------------------------------------------- selector
+
+def _select_check(Q, K, shape, C, I, Bk, rows_check=None):
+    cfg = abatt.Config(kv_block=Bk, clusters=C, kmeans_iters=I)
+    p, cent, sizes = abatt.select(Q.cuda(), K.cuda(), cfg, want_centroids=True)
+    p, cent, sizes = p.cpu().numpy(), cent.cpu().numpy(), sizes.cpu().numpy()
+    rows = _rows_of(shape) if rows_check is None else np.asarray(rows_check)
+    ocent, osz, _ = oracle.kmeans(Q, shape, rows, C, I)
+    same_sizes = np.all(sizes[rows] == osz, axis=1)
+    assert same_sizes.mean() >= 0.95
+    ok = same_sizes
+    assert np.max(np.abs(cent[rows][ok] - ocent[ok])) <= 1e-4 * max(1.0, np.abs(ocent).max())
+    p64, p32 = oracle.block_probs(Q, K, shape, rows, C, I, Bk=Bk)
+    assert np.allclose(p.sum(1), 1.0, atol=2e-4)
+    l1 = np.abs(p[rows][ok] - p64[ok]).sum(1)
+    assert np.max(l1) <= 2e-3, np.max(l1)
+    return p
+
+
+def test_select_tiny():
+    w = synth.TINY
+    Q, K, V = synth.generate(w)
+    _select_check(Q, K, w.shape, w.clusters, w.iters, w.Bk)
+
+
+@pytest.mark.parametrize("Bk,C", [(16, 8), (32, 3), (128, 16), (64, 1)])
+def test_select_d128_ragged(Bk, C):
+    w = synth.WAN_1_3B.with_(H=2, N=1000, grid=(1, 20, 50))
+    Q, K, V = synth.generate(w)
+    _select_check(Q, K, w.shape, C, 5, Bk)
+
+
+# ------------------------------------------------------------------------- end to end
+
+def _forward_check(w, rows_check, heads=None):
+    Q, K, V = synth.generate(w, heads=heads)
+    shape = (Q.shape[0], Q.shape[1], w.N, w.d)
+    cfg = cfg_of(w)
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, shape, cfg), dtype=torch.uint8,
+                     device="cuda")
+    O = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg, workspace=ws)
+    torch.cuda.synchronize()
+    assert abatt.read_status(ws) == 0
+    p, counts, idx, logw = (t.cpu().numpy() for t in abatt.intermediates(ws, shape, cfg))
+    # properties on every row
+    assert np.allclose(p.sum(1), 1.0, atol=2e-4)
+    M = oracle.budget_blocks(w.budget_bp, w.nK)
+    assert abs(counts.mean() - M) <= 4 * np.sqrt(M / len(counts)) + 1
+    for r in range(0, len(counts), max(1, len(counts) // 64)):
+        L = counts[r]
+        assert np.all(np.diff(idx[r, :L]) > 0) and idx[r, :L].min() >= 0 and idx[r, L - 1] < w.nK
+        assert np.all(logw[r, :L] >= 0)
+    # sampled rows against the oracle
+    rows = np.asarray(rows_check)
+    ref = oracle.forward(Q, K, V, shape, rows, w.clusters, w.iters, w.budget_bp, w.seed, Bk=w.Bk)
+    agree = agreement(counts[rows], idx[rows], ref["counts"], ref["idx"])
+    assert agree >= AGREE, agree
+    # the kernel on its own lists
+    o5, _ = oracle.ht_attention(Q, K, V, shape, rows, counts[rows], idx[rows], logw[rows], Bk=w.Bk)
+    Oc = O.float().cpu().numpy()
+    nQ = w.nQ
+    got = np.zeros_like(o5)
+    for k, r in enumerate(rows):
+        bh, q = divmod(int(r), nQ)
+        n = min(128, w.N - q * 128)
+        got[k, :n] = Oc[bh // shape[1], bh % shape[1], q * 128:q * 128 + n]
+    assert _rel_l2(got, o5) <= REL_L2
+    assert np.max(np.abs(got - o5)) <= MAX_ABS
+    return agree
+
+
+def test_forward_tiny_full():
+    w = synth.TINY
+    _forward_check(w, _rows_of(w.shape))
+
+
+def test_forward_wan1_3b_sampled_rows():
+    w = synth.WAN_1_3B
+    heads = 3
+    nQ = w.nQ
+    rows = [h * nQ + i for h in range(heads) for i in list(range(0, nQ, 32)) + [nQ - 1]]
+    _forward_check(w, rows, heads=heads)
+
+
+def test_forward_wan14b_full_size_sampled_rows():
+    w = synth.WAN_14B
+    nQ = w.nQ
+    rows = [h * nQ + i for h, i in [(0, 0), (0, nQ - 1), (7, 100), (13, 295), (21, 1), (27, 400),
+                                    (33, 590), (39, 0), (39, 333), (39, nQ - 1)]]
+    _forward_check(w, rows)
