@@ -229,6 +229,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with Clocks(local) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed region
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         start.record(stream)

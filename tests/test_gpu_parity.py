@@ -117,8 +117,12 @@ def test_sample_repeatable_on_other_stream():
     with torch.cuda.stream(s):
         b = abatt.sample(p, shape, cfg, stream=s)
     s.synchronize()
-    for x, y in zip(a[:3], b[:3]):
-        assert torch.equal(x, y)
+    assert torch.equal(a[0], b[0])
+    c = a[0].cpu().numpy()
+    for x, y in zip(a[1:3], b[1:3]):
+        x, y = x.cpu().numpy(), y.cpu().numpy()
+        for r in range(len(c)):
+            assert np.array_equal(x[r, :c[r]].view(np.uint32), y[r, :c[r]].view(np.uint32))
 
 
 # -------------------------------------------------------------------------- attention
@@ -192,9 +196,10 @@ def test_attention_keep_all_is_dense():
 
 def test_attention_large_logweights_and_scale():
     shape = (1, 1, 2048, 128)
-    Q, K, V = (synth.random_bf16(shape, s, 2.0) for s in (7, 8, 9))
-    rows, c, i, lw = _random_lists(shape, 16, 300, 23, conc=0.02)  # tiny pi -> large weights
-    assert lw.max() > 5
+    Q, K = (synth.random_bf16(shape, s, 2.0) for s in (7, 8))
+    V = synth.random_bf16(shape, 9)
+    rows, c, i, lw = _random_lists(shape, 16, 300, 23, conc=0.02)  # small pi -> large weights
+    assert lw.max() > 3
     _attn_check(Q, K, V, shape, 16, rows, c, i, lw, scale=0.2)
 
 
