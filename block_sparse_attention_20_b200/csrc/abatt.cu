@@ -50,9 +50,12 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
 // ---- workspace layout ----------------------------------------------------------
 struct Layout {
     size_t hdr, cent_hi, cent_lo, weight, r, mref, mz;  // select
+    size_t ulen, ublk, ulw;                               // attention (pair unions)
     size_t p, counts, idx, logw;                          // forward
     size_t total;
 };
+
+int64_t pairs_of(const Geom &g) { return g.heads * pairs_per_head(g.nQ); }
 
 Layout layout(abatt_call call, const Geom &g) {
     Layout L;
@@ -68,6 +71,12 @@ Layout layout(abatt_call call, const Geom &g) {
         L.r = off;       off = align256(off + crow * g.ldr * 4);
         L.mref = off;    off = align256(off + crow * g.nT * 4);
         L.mz = off;      off = align256(off + crow * 8);
+    }
+    if (call == ABATT_CALL_ATTENTION || call == ABATT_CALL_FORWARD) {
+        const size_t pairs = (size_t)pairs_of(g);
+        L.ulen = off; off = align256(off + pairs * 4);
+        L.ublk = off; off = align256(off + pairs * g.nK * 4);
+        L.ulw = off;  off = align256(off + pairs * 2 * g.nK * 4);
     }
     if (call == ABATT_CALL_FORWARD) {
         L.p = off;      off = align256(off + (size_t)g.rows * g.nK * 4);
@@ -127,6 +136,17 @@ bool make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t out
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D bf16 map with 128-byte swizzle and a 64-element inner box.
+bool make_map4(CUtensorMap *m, const void *base, const cuuint64_t dims[4],
+               const cuuint64_t strides[3], const cuuint32_t box[4]) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -201,17 +221,41 @@ abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, 
 
 abatt_status run_attention(const void *Q, const void *K, const void *V, const Geom &g,
                            const abatt_config *cfg, const int32_t *counts, const int32_t *idx,
-                           const float *logw, int capacity, void *O, float *lse, WsHeader *hdr,
-                           int sms, cudaStream_t st) {
+                           const float *logw, int capacity, void *O, float *lse, void *ws,
+                           const Layout &L, int sms, cudaStream_t st) {
+    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+    PairArgs pa;
+    pa.rows = g.rows; pa.pairs = pairs_of(g); pa.nQ = g.nQ; pa.nK = g.nK; pa.capacity = capacity; pa.cap_u = g.nK;
+    pa.counts = counts; pa.idx = idx; pa.logw = logw;
+    pa.ulen = at<int32_t>(ws, L.ulen);
+    pa.ublk = at<int32_t>(ws, L.ublk);
+    pa.ulw = at<float>(ws, L.ulw);
+    pa.status = &hdr->status;
+    if (launch_pair_union(pa, sms, st) != cudaSuccess) return ABATT_ERR_CUDA;
+
+    const int CH = g.d / 64;
+    const bool fold = (g.N % 8) == 0 && g.heads * (g.N / 8) < (int64_t(1) << 31);
     AttnMaps m;
-    if (!make_map(&m.q, Q, g.d, g.N, g.heads, 128) || !make_map(&m.k, K, g.d, g.N, g.heads, g.Bk) ||
-        !make_map(&m.v, V, g.d, g.N, g.heads, g.Bk))
+    if (!make_map(&m.q, Q, g.d, g.N, g.heads, 128)) return ABATT_ERR_CUDA;
+    if (fold) {
+        const cuuint64_t dims[4] = {64, 8, (cuuint64_t)CH, (cuuint64_t)(g.heads * (g.N / 8))};
+        const cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, 128, (cuuint64_t)8 * g.d * 2};
+        const cuuint32_t box[4] = {64, 8, (cuuint32_t)CH, (cuuint32_t)(g.Bk / 8)};
+        if (!make_map4(&m.k, K, dims, strides, box)) return ABATT_ERR_CUDA;
+    } else if (!make_map(&m.k, K, g.d, g.N, g.heads, g.Bk)) {
         return ABATT_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[4] = {64, (cuuint64_t)g.N, (cuuint64_t)CH, (cuuint64_t)g.heads};
+        const cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, 128, (cuuint64_t)g.N * g.d * 2};
+        const cuuint32_t box[4] = {64, (cuuint32_t)g.Bk, (cuuint32_t)CH, 1};
+        if (!make_map4(&m.v, V, dims, strides, box)) return ABATT_ERR_CUDA;
+    }
     AttnArgs a;
-    a.rows = g.rows; a.nQ = g.nQ; a.N = g.N; a.D = g.d; a.Bk = g.Bk; a.nK = g.nK;
-    a.capacity = capacity;
+    a.rows = g.rows; a.pairs = pairs_of(g); a.nQ = g.nQ; a.N = g.N; a.D = g.d; a.Bk = g.Bk;
+    a.nK = g.nK; a.cap_u = g.nK; a.k_fold = fold ? 1 : 0;
     a.scale_log2 = cfg->scale * kLog2eF;
-    a.counts = counts; a.idx = idx; a.logw = logw;
+    a.ulen = pa.ulen; a.ublk = pa.ublk; a.ulw = pa.ulw;
     a.O = static_cast<__nv_bfloat16 *>(O);
     a.lse = lse;
     a.hdr = hdr;
@@ -301,9 +345,10 @@ abatt_status abatt_attention(const void *Q, const void *K, const void *V,
     int sms = 0;
     if ((s = device_sms(&sms)) != ABATT_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Layout L = layout(ABATT_CALL_ATTENTION, g);
     if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
-    return run_attention(Q, K, V, g, cfg, counts, idx, logw, capacity, O, lse,
-                         static_cast<WsHeader *>(workspace), sms, st);
+    return run_attention(Q, K, V, g, cfg, counts, idx, logw, capacity, O, lse, workspace, L, sms,
+                         st);
 }
 
 abatt_status abatt_forward(const void *Q, const void *K, const void *V,
@@ -329,7 +374,7 @@ abatt_status abatt_forward(const void *Q, const void *K, const void *V,
     if ((s = run_select(Q, K, g, cfg, p, nullptr, nullptr, workspace, L, sms, st)) != ABATT_OK)
         return s;
     if ((s = run_sample(p, g, cfg, counts, idx, logw, g.nK, hdr, sms, st)) != ABATT_OK) return s;
-    return run_attention(Q, K, V, g, cfg, counts, idx, logw, g.nK, O, lse, hdr, sms, st);
+    return run_attention(Q, K, V, g, cfg, counts, idx, logw, g.nK, O, lse, workspace, L, sms, st);
 }
 
 abatt_status abatt_forward_intermediates(void *workspace, const abatt_shape *shape,

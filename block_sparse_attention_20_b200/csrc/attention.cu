@@ -4,99 +4,196 @@
 // sentence: each drawn block is re-weighted by 1/pi, here as +ln(1/pi) on
 // its logits inside the online softmax).
 //
-// One CTA per query block (128 queries).  Warp roles:
-//   warp 0     TMA: Q once; then, per 128-key tile, 128/Bk boxes of Bk rows of
-//              K and of V, each landing at its slot of a 128-row 128-byte-
-//              swizzled tile (empty slots of the last tile are filled with
-//              zeros by loading a box past the end of the tensor);
-//   warp 1     tcgen05 MMA issuer: S = Q K^T into a double-buffered 128x128
-//              fp32 accumulator in tensor memory, O += P V into a 128xD fp32
-//              accumulator in tensor memory;
-//   warps 2-5  softmax (thread = query row): base-2 logits plus the block's
-//              log-weight, running maximum with a lazy rescale threshold,
-//              P in bf16 to shared memory, O correction in tensor memory,
-//              final normalisation and bf16 store.
+// B200 design.  On this GPU the kernel is bound by how fast gathered K/V
+// bytes move from L2 to the SMs, not by the tensor cores, so neighbouring
+// query blocks share their gathers:
+//
+//   pair_union_kernel   rows 2p and 2p+1 (a "pair") get one ascending union
+//                       of their two drawn lists, with each row's log-weight
+//                       per union block (-1 where the row did not draw it).
+//   gather_attn_kernel  persistent, one CTA per SM, one pair at a time.  Each
+//                       128-key tile of the union is gathered once (one 4 KB
+//                       TMA box per 16-key block for K and for V) and used by
+//                       both rows; a row gives the blocks it did not draw a
+//                       -inf logit, so they add exactly zero.
+//
+//   tensor core, per tile t:   S0(t)  PV1(t-1)  S1(t)  PV0(t)
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q of both rows, then K(t), V(t) into a ring;
+//   warp 1      tensor-memory owner and tcgen05 MMA issuer:
+//               S_s = Q_s K^T (fp32, 128 TMEM columns per row),
+//               O_s += P_s V  (P_s read back from the columns S_s used);
+//   warps 2-3   idle;
+//   warps 4-7   softmax of row 0, warps 8-11 softmax of row 1 (thread = query):
+//               one TMEM read of the tile, raw per-block maxima, tile maximum
+//               of s*log2(e)*S + log-weight (base 2), lazy running maximum
+//               (O is rescaled only when it grows by more than 8), P in bf16
+//               back into tensor memory chunk by chunk, final O / l to bf16.
 #include "kernels.cuh"
 
 namespace abatt {
 
 namespace {
 
-constexpr int kAttnThreads = 192;
-constexpr int kKStages = 2;
-constexpr int kVStages = 2;
+constexpr int kAttnThreads = 384;
 #define kNegInf (-__int_as_float(0x7f800000))
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;  // base-2: values up to 2^8 stay in fp32/bf16 range
+constexpr float kRescaleThreshold = 8.0f;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int D, int BK>
+// ============================== pair union ======================================
+constexpr int kUnionThreads = 256;
+
+// Entry j of a list is used if it is a block index and exceeds the previous
+// entry (when that one is a block index itself).
+__device__ __forceinline__ bool union_entry_ok(const int32_t *idx, int j, int k, int nK) {
+    if (k < 0 || k >= nK) return false;
+    if (j == 0) return true;
+    const int prev = idx[j - 1];
+    return prev < 0 || prev >= nK || prev < k;
+}
+
+__global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArgs a) {
+    // [W] membership bitmap of each row, [W] union prefix (exclusive) per word
+    extern __shared__ uint32_t sm_union[];
+    __shared__ int32_t wsum[kUnionThreads / 32];
+    const int W = (a.nK + 31) >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t *bA = sm_union, *bB = sm_union + W, *pre = sm_union + 2 * W;
+    for (int64_t pr = blockIdx.x; pr < a.pairs; pr += gridDim.x) {
+        __syncthreads();
+        for (int w = tid; w < 2 * W; w += kUnionThreads) sm_union[w] = 0;
+        __syncthreads();
+        int64_t rr[2];
+        pair_rows(pr, a.nQ, &rr[0], &rr[1]);
+        int L[2];
+        bool bad = false;
+        for (int s = 0; s < 2; ++s) {
+            L[s] = rr[s] >= 0 ? min(max(a.counts[rr[s]], 0), a.capacity) : 0;
+            const int32_t *idx = a.idx + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
+            uint32_t *b = s ? bB : bA;
+            for (int j = tid; j < L[s]; j += kUnionThreads) {
+                const int k = idx[j];
+                if (!union_entry_ok(idx, j, k, a.nK)) { bad = true; continue; }
+                atomicOr(&b[k >> 5], 1u << (k & 31));
+            }
+        }
+        if (__syncthreads_or(bad) && tid == 0) raise_flag(a.status, ABATT_DEVFLAG_BADLIST);
+        // exclusive prefix of the union's popcount per word: each thread owns a
+        // contiguous run of words, block-wide scan of the run totals
+        const int per = (W + kUnionThreads - 1) / kUnionThreads;
+        const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(bA[w] | bB[w]);
+        int x = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[warp] = x;
+        __syncthreads();
+        int run = x - cnt, total = 0;
+        for (int w = 0; w < kUnionThreads / 32; ++w) {
+            if (w < warp) run += wsum[w];
+            total += wsum[w];
+        }
+        for (int w = w0; w < w1; ++w) {
+            pre[w] = run;
+            run += __popc(bA[w] | bB[w]);
+        }
+        __syncthreads();
+        int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
+        float *uw = a.ulw + pr * 2 * (int64_t)a.cap_u;
+        // union block ids in ascending order; both log-weights start as "not drawn"
+        for (int w = tid; w < W; w += kUnionThreads) {
+            uint32_t mu = bA[w] | bB[w];
+            int pos = pre[w];
+            while (mu) {
+                const int bit = __ffs(mu) - 1;
+                mu &= mu - 1;
+                if (pos < a.cap_u) {
+                    ub[pos] = w * 32 + bit;
+                    uw[pos] = -1.0f;
+                    uw[a.cap_u + pos] = -1.0f;
+                }
+                ++pos;
+            }
+        }
+        __syncthreads();
+        // each valid drawn entry writes its log-weight at its union position
+        for (int s = 0; s < 2; ++s) {
+            const int32_t *idx = a.idx + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
+            const float *lw = a.logw + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
+            for (int j = tid; j < L[s]; j += kUnionThreads) {
+                const int k = idx[j];
+                if (!union_entry_ok(idx, j, k, a.nK)) continue;
+                const uint32_t mu = bA[k >> 5] | bB[k >> 5];
+                const int pos = pre[k >> 5] + __popc(mu & ((1u << (k & 31)) - 1u));
+                if (pos < a.cap_u) uw[s * a.cap_u + pos] = lw[j];
+            }
+        }
+        if (tid == 0) a.ulen[pr] = min(total, a.cap_u);
+    }
+}
+
+// ============================== attention ======================================
+template <int D>
+struct AttnCfg {
+    static constexpr int CH = D / 64;
+    static constexpr uint32_t TILE = 128u * D * 2u;
+    static constexpr int ST = D == 128 ? 5 : 10;  // K/V ring stages
+    static constexpr size_t SMEM = (size_t)(2 + ST) * TILE + 1024;
+};
+
+template <int D, int BK, bool KFOLD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     gather_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a) {
-    constexpr int CH = D / 64;
-    constexpr uint32_t TILE = 128u * D * 2u;  // a 128-row operand tile
-    constexpr int BPT = 128 / BK;             // blocks per 128-key tile
-    constexpr uint32_t TMEM_COLS = 512;       // S0 | S1 | O
-    constexpr uint32_t O_COL = 256;
+    using Cfg = AttnCfg<D>;
+    constexpr int CH = Cfg::CH;
+    constexpr uint32_t TILE = Cfg::TILE;
+    constexpr int ST = Cfg::ST;
+    constexpr int BPT = 128 / BK;
+    constexpr uint32_t BLK = (uint32_t)BK * D * 2;  // bytes of one gathered block
+    constexpr uint32_t TMEM_COLS = 512;             // S0 | S1 | O0 | O1
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *sQ = smem;
-    uint8_t *sK = sQ + TILE;
-    uint8_t *sV = sK + kKStages * TILE;
-    uint8_t *sP = sV + kVStages * TILE;
+    uint8_t *sQ = smem;                // [2][TILE]
+    uint8_t *sRing = smem + 2 * TILE;  // [ST][TILE]
 
-    __shared__ __align__(8) uint64_t bar_q, bar_p, bar_pv;
-    __shared__ __align__(8) uint64_t bar_kf[kKStages], bar_ke[kKStages];
-    __shared__ __align__(8) uint64_t bar_vf[kVStages], bar_ve[kVStages];
-    __shared__ __align__(8) uint64_t bar_sf[2], bar_se[2];
+    __shared__ __align__(8) uint64_t bar_qf[2], bar_qe[2];
+    __shared__ __align__(8) uint64_t bar_kvf[ST], bar_kve[ST];
+    __shared__ __align__(8) uint64_t bar_sf[2], bar_pf[2], bar_of[2], bar_oe[2];
+    __shared__ __align__(8) uint64_t bar_drain;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.x;
-    const int i = (int)(row % a.nQ);
-    const int hd = (int)(row / a.nQ);
-    const int nrows = min(128, a.N - i * 128);
-    const int L = min(max(a.counts[row], 0), a.capacity);
-    const int ntiles = (L + BPT - 1) / BPT;
-    const int32_t *idx = a.idx + row * (int64_t)a.capacity;
-    const float *lw = a.logw + row * (int64_t)a.capacity;
-    const int64_t tok0 = (int64_t)hd * a.N + (int64_t)i * 128;
-
-    // a bounded wait elsewhere already gave up: do not start more work
     if (a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT))
-        return;
-    if (L == 0) {  // empty list: O = 0, lse = -inf
-        for (int e = threadIdx.x; e < nrows * D / 8; e += blockDim.x)
-            reinterpret_cast<uint4 *>(a.O + tok0 * D)[e] = make_uint4(0, 0, 0, 0);
-        if (a.lse)
-            for (int r = threadIdx.x; r < nrows; r += blockDim.x) a.lse[tok0 + r] = kNegInf;
-        return;
-    }
-
+        return;  // a bounded wait elsewhere already gave up: start no more work
     const WaitCtx wc{&abort_s, a.hdr, a.wait_ns};
+
     if (threadIdx.x == 0) {
         abort_s = 0;
-        mbar_init(&bar_q, 1);
-        mbar_init(&bar_p, 4);
-        mbar_init(&bar_pv, 1);
-        for (int s = 0; s < kKStages; ++s) {
-            mbar_init(&bar_kf[s], 1);
-            mbar_init(&bar_ke[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar_qf[s], 1);
+            mbar_init(&bar_qe[s], 1);
+            mbar_init(&bar_sf[s], 1);
+            mbar_init(&bar_pf[s], 4);
+            mbar_init(&bar_of[s], 1);
+            mbar_init(&bar_oe[s], 4);
         }
-        for (int s = 0; s < kVStages; ++s) {
-            mbar_init(&bar_vf[s], 1);
-            mbar_init(&bar_ve[s], 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&bar_kvf[s], 1);
+            mbar_init(&bar_kve[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&bar_sf[b], 1);
-            mbar_init(&bar_se[b], 4);
-        }
+        mbar_init(&bar_drain, 1);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -108,246 +205,325 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
 
-    int k_issued = 0, v_issued = 0;  // TMA role bookkeeping for the drain
-    int committed = 0;               // MMA role: PV tiles committed
+    uint32_t ring_issued = 0;  // producer: ring loads issued (for the drain)
 
     if (warp == 0) {
-        // ------------------------------ TMA gather --------------------------------
+        // ================================ TMA producer ================================
+        // The whole warp: lane 0 owns the barriers; lane k < 128/Bk gathers
+        // block k of each tile, its index prefetched one tile ahead.
         if (lane == 0) {
             tma_prefetch_desc(&maps.q);
             tma_prefetch_desc(&maps.k);
             tma_prefetch_desc(&maps.v);
-            mbar_arrive_expect_tx(&bar_q, TILE);
-            for (int c = 0; c < CH; ++c)
-                tma_load_3d(sQ + c * 16384, &maps.q, &bar_q, c * 64, i * 128, hd);
-            const int pad_y = a.nK * BK;  // a box starting here lies wholly past N
-            bool bad = false;
-            for (int t = 0; t <= ntiles; ++t) {
-                if (t < ntiles) {
-                    const int s = t % kKStages;
-                    if (t >= kKStages && !mbar_wait(&bar_ke[s], ((t / kKStages) - 1) & 1, wc, 0x201))
+        }
+        const int groups_per_head = a.N / 8;
+        uint32_t q_loads[2] = {0, 0};
+        uint32_t rp = 0;
+        bool ok = true;
+        for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
+            const int U = a.ulen[pr];
+            const int n = (U + BPT - 1) / BPT;
+            if (n == 0) continue;
+            int64_t rr[2];
+            pair_rows(pr, a.nQ, &rr[0], &rr[1]);
+            const int hd = (int)(rr[0] / a.nQ);
+            const int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
+            int nxt = (lane < BPT && lane < U) ? __ldg(ub + lane) : -1;
+            if (lane == 0) {
+                for (int s = 0; s < 2; ++s) {
+                    const int64_t row = rr[s];
+                    if (row < 0) continue;
+                    if (q_loads[s] > 0 && !mbar_wait(&bar_qe[s], (q_loads[s] - 1) & 1, wc, 0x202)) {
+                        ok = false;
                         break;
-                    mbar_arrive_expect_tx(&bar_kf[s], TILE);
-                    for (int k = 0; k < BPT; ++k) {
-                        const int sidx = t * BPT + k;
-                        int y = pad_y;
-                        if (sidx < L) {
-                            const int b = idx[sidx];
-                            if (b >= 0 && b < a.nK) y = b * BK; else bad = true;
-                        }
-                        for (int c = 0; c < CH; ++c)
-                            tma_load_3d(sK + s * TILE + c * 16384 + k * BK * 128, &maps.k, &bar_kf[s],
-                                        c * 64, y, hd);
                     }
-                    k_issued = t + 1;
-                }
-                if (t >= 1) {
-                    const int tv = t - 1, s = tv % kVStages;
-                    if (tv >= kVStages && !mbar_wait(&bar_ve[s], ((tv / kVStages) - 1) & 1, wc, 0x202))
-                        break;
-                    mbar_arrive_expect_tx(&bar_vf[s], TILE);
-                    for (int k = 0; k < BPT; ++k) {
-                        const int sidx = tv * BPT + k;
-                        int y = pad_y;
-                        if (sidx < L) {
-                            const int b = idx[sidx];
-                            if (b >= 0 && b < a.nK) y = b * BK;
-                        }
-                        for (int c = 0; c < CH; ++c)
-                            tma_load_3d(sV + s * TILE + c * 16384 + k * BK * 128, &maps.v, &bar_vf[s],
-                                        c * 64, y, hd);
-                    }
-                    v_issued = tv + 1;
+                    mbar_arrive_expect_tx(&bar_qf[s], TILE);
+                    const int i = (int)(row % a.nQ), h = (int)(row / a.nQ);
+                    for (int c = 0; c < CH; ++c)
+                        tma_load_3d(sQ + s * TILE + c * 16384, &maps.q, &bar_qf[s], c * 64, i * 128, h);
+                    ++q_loads[s];
                 }
             }
-            if (bad) raise_flag(a.hdr ? &a.hdr->status : nullptr, ABATT_DEVFLAG_BADLIST);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            for (int t = 0; ok && t < n; ++t) {
+                const int blk = nxt;
+                const int jn = (t + 1) * BPT + lane;
+                nxt = (lane < BPT && jn < U) ? __ldg(ub + jn) : -1;
+                for (int kv = 0; kv < 2; ++kv) {  // K(t) then V(t)
+                    const int stg = rp % ST;
+                    if (lane == 0) {
+                        if (rp >= ST && !mbar_wait(&bar_kve[stg], ((rp / ST) - 1) & 1, wc, 0x201)) ok = false;
+                        if (ok) mbar_arrive_expect_tx(&bar_kvf[stg], TILE);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    if (lane < BPT) {
+                        uint8_t *dst = sRing + stg * TILE;
+                        const bool valid = blk >= 0;
+                        if (kv == 0) {
+                            if (KFOLD) {
+                                // groups of 8 rows with all heads folded: a box of Bk/8 groups
+                                const int g = valid ? hd * groups_per_head + blk * (BK / 8) : 0x7fffff00;
+                                tma_load_4d(dst + lane * BLK, &maps.k, &bar_kvf[stg], 0, 0, 0, g);
+                            } else {
+                                const int y = valid ? blk * BK : a.nK * BK;
+                                for (int c = 0; c < CH; ++c)
+                                    tma_load_3d(dst + c * 16384 + lane * BK * 128, &maps.k, &bar_kvf[stg],
+                                                c * 64, y, hd);
+                            }
+                        } else {
+                            const int y = valid ? blk * BK : a.nK * BK;
+                            tma_load_4d(dst + lane * BLK, &maps.v, &bar_kvf[stg], 0, y, 0, hd);
+                        }
+                    }
+                    ++rp;
+                    if (lane == 0) ring_issued = rp;
+                }
+            }
         }
     } else if (warp == 1) {
-        // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0 && mbar_wait(&bar_q, 0, wc, 0x203)) {
+        // ================================ MMA issuer ==================================
+        if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(128, 128);
             constexpr uint32_t idesc_o = idesc_bf16(128, D, /*b_mn_major=*/true);
-            const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-            auto issue_s = [&](int t) -> bool {
-                const int s = t % kKStages, buf = t & 1;
-                if (!mbar_wait(&bar_kf[s], (t / kKStages) & 1, wc, 0x204)) return false;
-                if (t >= 2 && !mbar_wait(&bar_se[buf], ((t >> 1) - 1) & 1, wc, 0x205)) return false;
+            uint32_t rp = 0;  // ring position of K(t); V(t) is rp+1
+            uint32_t q_uses[2] = {0, 0}, pv_ops[2] = {0, 0}, o_items[2] = {0, 0};
+            bool ok = true;
+            const uint32_t q_addr0 = smem_u32(sQ), ring_addr = smem_u32(sRing);
+            auto op_s = [&](int s, uint32_t kpos, bool release, bool last) -> bool {
+                const int stg = kpos % ST;
+                if (!mbar_wait(&bar_kvf[stg], (kpos / ST) & 1, wc, 0x203)) return false;
                 tc_fence_after();
-                const uint32_t k_addr = smem_u32(sK + s * TILE);
+                const uint32_t qa = q_addr0 + s * TILE, ka = ring_addr + stg * TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_bf16_ss(tmem + buf * 128, sdesc_sw128(q_addr + off, 16, 1024),
-                                 sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0);
+                    const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint32_t koff =
+                        KFOLD ? (kk >> 2) * 1024 + (kk & 3) * 32 : (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_bf16_ss(tmem + s * 128, sdesc_sw128(qa + qoff, 16, 1024),
+                                 sdesc_sw128(ka + koff, 16, KFOLD ? CH * 1024 : 1024), idesc_s, kk > 0);
                 }
-                umma_commit(&bar_ke[s]);
-                umma_commit(&bar_sf[buf]);
+                if (release) umma_commit(&bar_kve[stg]);
+                umma_commit(&bar_sf[s]);
+                if (last) umma_commit(&bar_qe[s]);
                 return true;
             };
-            tc_fence_after();
-            bool ok = issue_s(0);
-            for (int t = 0; ok && t < ntiles; ++t) {
-                if (t + 1 < ntiles && !issue_s(t + 1)) break;
-                const int s = t % kVStages;
-                if (!mbar_wait(&bar_p, t & 1, wc, 0x206)) break;
-                if (!mbar_wait(&bar_vf[s], (t / kVStages) & 1, wc, 0x207)) break;
+            auto op_pv = [&](int s, uint32_t vpos, int t, bool release, bool last) -> bool {
+                if (!mbar_wait(&bar_pf[s], pv_ops[s] & 1, wc, 0x204)) return false;
+                if (t == 0 && o_items[s] > 0 &&
+                    !mbar_wait(&bar_oe[s], (o_items[s] - 1) & 1, wc, 0x205))
+                    return false;
+                const int stg = vpos % ST;
+                if (!mbar_wait(&bar_kvf[stg], (vpos / ST) & 1, wc, 0x206)) return false;
                 tc_fence_after();
-                const uint32_t v_addr = smem_u32(sV + s * TILE);
+                const uint32_t va = ring_addr + stg * TILE;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t adesc = sdesc_sw128(p_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, 16384, 1024);
-                    umma_bf16_ss(tmem + O_COL, adesc, bdesc, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t boff = (uint32_t)((16 * j) / BK) * BLK + (uint32_t)((16 * j) % BK) * 128;
+                    umma_bf16_ts(tmem + 256 + s * 128, tmem + s * 128 + j * 8,
+                                 sdesc_sw128(va + boff, BK * 128, 1024), idesc_o,
+                                 (t > 0 || j > 0) ? 1u : 0u);
                 }
-                umma_commit(&bar_ve[s]);
-                umma_commit(&bar_pv);
-                committed = t + 1;
+                if (release) umma_commit(&bar_kve[stg]);
+                if (last) {
+                    umma_commit(&bar_of[s]);
+                    ++o_items[s];
+                }
+                ++pv_ops[s];
+                return true;
+            };
+            for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
+                const int U = a.ulen[pr];
+                const int n = (U + BPT - 1) / BPT;
+                if (n == 0) continue;
+                int64_t rr[2];
+                pair_rows(pr, a.nQ, &rr[0], &rr[1]);
+                const bool has1 = rr[1] >= 0;
+                for (int s = 0; ok && s < (has1 ? 2 : 1); ++s) {
+                    if (!mbar_wait(&bar_qf[s], q_uses[s] & 1, wc, 0x207)) ok = false;
+                    ++q_uses[s];
+                }
+                const uint32_t base = rp;
+                for (int t = 0; ok && t <= n; ++t) {
+                    const uint32_t kp = base + 2 * t, vp_prev = base + 2 * (t - 1) + 1, vp = kp + 1;
+                    if (t < n && !op_s(0, kp, !has1, t == n - 1)) ok = false;
+                    if (ok && has1 && t >= 1 && !op_pv(1, vp_prev, t - 1, true, t - 1 == n - 1)) ok = false;
+                    if (ok && has1 && t < n && !op_s(1, kp, true, t == n - 1)) ok = false;
+                    if (ok && t < n && !op_pv(0, vp, t, !has1, t == n - 1)) ok = false;
+                }
+                rp = base + 2 * n;
             }
         }
-    } else {
-        // ------------------------------ softmax -----------------------------------
-        const int wq = warp & 3;
-        const int r = wq * 32 + lane;  // query row == TMEM lane
+    } else if (warp >= 4) {
+        // ================================ softmax =====================================
+        const int s = (warp - 4) >> 2;  // row of the pair
+        const int wq = warp & 3;        // tensor-memory lane quarter
+        const int r = wq * 32 + lane;   // query row within the block == TMEM lane
         const uint32_t t_lane = (uint32_t)(wq * 32) << 16;
-        float m_run = kNegInf, l = 0.0f;
+        const uint32_t s_col = tmem + t_lane + s * 128;
+        const uint32_t o_col = tmem + t_lane + 256 + s * 128;
+        uint32_t s_uses = 0, o_uses = 0;
         bool ok = true;
-        for (int t = 0; t < ntiles; ++t) {
-            // per-slot bias (log-weight in base 2, or -inf) and valid key count
-            float bias[BPT];
-            int keep[BPT];
+        for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
+            int64_t rr[2];
+            pair_rows(pr, a.nQ, &rr[0], &rr[1]);
+            const int64_t row = rr[s];
+            if (row < 0) continue;  // the pair's second row does not exist
+            const int U = a.ulen[pr];
+            const int n = (U + BPT - 1) / BPT;
+            const int i = (int)(row % a.nQ), hd = (int)(row / a.nQ);
+            const int nrows = min(128, a.N - i * 128);
+            const int64_t tok = (int64_t)hd * a.N + (int64_t)i * 128 + r;
+            const int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
+            const float *lw = a.ulw + (pr * 2 + s) * (int64_t)a.cap_u;
+            float m_run = kNegInf, l = 0.0f;
+            for (int t = 0; t < n; ++t) {
+                // per-block base-2 log-weight (-inf where this row did not draw
+                // the block or the slot is empty); the one block that can be
+                // cut by N is the last block of the sequence
+                float bias[BPT];
+                int tail_k = -1, tail_keep = BK;
 #pragma unroll
-            for (int k = 0; k < BPT; ++k) {
-                const int sidx = t * BPT + k;
-                bias[k] = kNegInf;
-                keep[k] = 0;
-                if (sidx < L) {
-                    const int b = idx[sidx];
-                    if (b >= 0 && b < a.nK) {
-                        bias[k] = lw[sidx] * kLog2e;
-                        keep[k] = min(BK, a.N - b * BK);
+                for (int k = 0; k < BPT; ++k) {
+                    const int j = t * BPT + k;
+                    bias[k] = kNegInf;
+                    if (j < U) {
+                        const float w = __ldg(lw + j);
+                        if (w >= 0.0f) bias[k] = w * kLog2e;
+                        const int b = __ldg(ub + j);
+                        if (b == a.nK - 1 && a.N - b * BK < BK) {
+                            tail_k = k;
+                            tail_keep = a.N - b * BK;
+                        }
                     }
                 }
-            }
-            const int buf = t & 1;
-            if (!mbar_wait(&bar_sf[buf], (t >> 1) & 1, wc, 0x208)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t v[4][32];
-            const uint32_t sa = tmem + t_lane + buf * 128;
-            tmem_ld32(sa + 0, v[0]);
-            tmem_ld32(sa + 32, v[1]);
-            tmem_ld32(sa + 64, v[2]);
-            tmem_ld32(sa + 96, v[3]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_se[buf]);
+                const bool masked = tail_k >= 0;
+                if (!mbar_wait(&bar_sf[s], s_uses & 1, wc, 0x208)) { ok = false; break; }
+                ++s_uses;
+                tc_fence_after();
 
-            float tmax = kNegInf;
+                uint32_t v[4][32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+                for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, v[c]);
+                tmem_wait_ld();
+                if (masked) {  // keys past N inside the last block of the sequence
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int col = q * 32 + c;
-                    float x = fmaf(__uint_as_float(v[q][c]), a.scale_log2, bias[col / BK]);
-                    if ((col % BK) >= keep[col / BK]) x = kNegInf;
-                    v[q][c] = __float_as_uint(x);
-                    tmax = fmaxf(tmax, x);
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if ((c * 32 + j) / BK == tail_k && (c * 32 + j) % BK >= tail_keep)
+                                v[c][j] = __float_as_uint(kNegInf);
                 }
-            const bool need = tmax > m_run + kRescaleThreshold;
-            const float m_use = need ? tmax : m_run;
-            const float alpha = need ? ((m_run == kNegInf) ? 0.0f : ex2_approx(m_run - tmax)) : 1.0f;
-            const float m_sub = (m_use == kNegInf) ? 0.0f : m_use;  // all-masked tile: p = 0
-            float rs = 0.0f;
-            uint32_t pk[64];
+                float bmax[BPT];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+                for (int k = 0; k < BPT; ++k) bmax[k] = kNegInf;
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float p0 = ex2_approx(__uint_as_float(v[q][c]) - m_sub);
-                    const float p1 = ex2_approx(__uint_as_float(v[q][c + 1]) - m_sub);
-                    rs += p0 + p1;
-                    pk[(q * 32 + c) >> 1] = pack_bf16x2(p0, p1);
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int k = (c * 32 + j) / BK;
+                        bmax[k] = fmaxf(bmax[k], __uint_as_float(v[c][j]));
+                    }
+                float tmax = kNegInf;
+#pragma unroll
+                for (int k = 0; k < BPT; ++k) tmax = fmaxf(tmax, fmaf(bmax[k], a.scale_log2, bias[k]));
+                const bool need = tmax > m_run + kRescaleThreshold;
+                const float m_use = need ? tmax : m_run;
+                const float alpha = need ? ((m_run == kNegInf) ? 0.0f : ex2_approx(m_run - tmax)) : 1.0f;
+                const float m_sub = (m_use == kNegInf) ? 0.0f : m_use;
+#pragma unroll
+                for (int k = 0; k < BPT; ++k) bias[k] -= m_sub;  // now the exponent offset
+                float rs = 0.0f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const int k0 = (c * 32 + j) / BK, k1 = (c * 32 + j + 1) / BK;
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c][j]), a.scale_log2, bias[k0]));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c][j + 1]), a.scale_log2, bias[k1]));
+                        rs += p0 + p1;
+                        pk[j >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(s_col + c * 16, pk);
                 }
-            l = fmaf(l, alpha, rs);
-            m_run = m_use;
-
-            // O and the P buffer are free once the previous PV has completed
-            if (t > 0 && !mbar_wait(&bar_pv, (t - 1) & 1, wc, 0x209)) { ok = false; break; }
-            tc_fence_after();
-            if (t > 0 && __any_sync(0xffffffffu, need)) {
+                // rescale O (after P, so the scores are dead): the commit that
+                // signalled S(t) covers the previous PV of this row
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t o[32];
-                    const uint32_t oa = tmem + t_lane + O_COL + q * 32;
-                    tmem_ld32(oa, o);
-                    tmem_wait_ld();
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_col + c * 32, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tmem_st32(oa, o);
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st32(o_col + c * 32, o);
+                    }
                 }
                 tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_pf[s]);
+                l = fmaf(l, alpha, rs);
+                m_run = m_use;
             }
-            // P row r, keys 0..127, into the two 64-key swizzled chunks
+            if (!ok) break;
+            __nv_bfloat16 *orow = a.O + tok * D;
+            if (n == 0) {  // no block at all: O = 0, lse = -inf
+                if (r < nrows) {
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int base = ch * 32 + u * 4;
-                    const uint4 val = make_uint4(pk[base], pk[base + 1], pk[base + 2], pk[base + 3]);
-                    *reinterpret_cast<uint4 *>(sP + ch * 16384 + r * 128 + ((u ^ (r & 7)) << 4)) = val;
+                    for (int q = 0; q < D / 8; ++q) reinterpret_cast<uint4 *>(orow)[q] = make_uint4(0, 0, 0, 0);
+                    if (a.lse) a.lse[tok] = kNegInf;
                 }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_p);
-        }
-        // epilogue: O / l -> bf16
-        if (ok && mbar_wait(&bar_pv, (ntiles - 1) & 1, wc, 0x20a)) {
+                continue;
+            }
+            // epilogue: O / l -> bf16, then release O to this slot's next row
+            if (!mbar_wait(&bar_of[s], o_uses & 1, wc, 0x209)) { ok = false; break; }
+            ++o_uses;
             tc_fence_after();
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            __nv_bfloat16 *orow = a.O + (tok0 + r) * D;
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tmem + t_lane + O_COL + q * 32, o);
+                tmem_ld32(o_col + c * 32, o);
                 tmem_wait_ld();
                 if (r < nrows) {
 #pragma unroll
-                    for (int c = 0; c < 32; c += 8) {
+                    for (int j = 0; j < 32; j += 8) {
                         uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[c + 0]) * inv, __uint_as_float(o[c + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(o[c + 2]) * inv, __uint_as_float(o[c + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(o[c + 4]) * inv, __uint_as_float(o[c + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(o[c + 6]) * inv, __uint_as_float(o[c + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow + q * 32 + c) = w;
+                        w.x = pack_bf16x2(__uint_as_float(o[j + 0]) * inv, __uint_as_float(o[j + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(o[j + 4]) * inv, __uint_as_float(o[j + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(o[j + 6]) * inv, __uint_as_float(o[j + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(orow + c * 32 + j) = w;
                     }
                 }
             }
-            if (a.lse && r < nrows) a.lse[tok0 + r] = (m_run + __log2f(l)) * kLn2;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_oe[s]);
+            if (a.lse && r < nrows) a.lse[tok] = l > 0.0f ? (m_run + __log2f(l)) * kLn2 : kNegInf;
         }
         tc_fence_before();
     }
 
-    // ------------------------------ teardown --------------------------------------
+    // ================================ teardown ========================================
     __syncthreads();
     if (abort_s) {
+        // let copies still in flight land before shared memory goes away
         if (warp == 0 && lane == 0) {
-            for (int t = k_issued - kKStages > 0 ? k_issued - kKStages : 0; t < k_issued; ++t) {
+            for (uint32_t q = ring_issued > ST ? ring_issued - ST : 0; q < ring_issued; ++q) {
                 const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(&bar_kf[t % kKStages], (t / kKStages) & 1) &&
-                       globaltimer_ns() - t0 < a.wait_ns) {
-                }
-            }
-            for (int t = v_issued - kVStages > 0 ? v_issued - kVStages : 0; t < v_issued; ++t) {
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(&bar_vf[t % kVStages], (t / kVStages) & 1) &&
+                while (!mbar_try_wait(&bar_kvf[q % ST], (q / ST) & 1) &&
                        globaltimer_ns() - t0 < a.wait_ns) {
                 }
             }
         }
-        if (warp == 1 && lane == 0 && committed > 0) {
+        // and MMAs: a commit issued now arrives once all earlier MMAs are done
+        if (warp == 1 && lane == 0) {
+            umma_commit(&bar_drain);
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&bar_pv, (committed - 1) & 1) && globaltimer_ns() - t0 < a.wait_ns) {
+            while (!mbar_try_wait(&bar_drain, 0) && globaltimer_ns() - t0 < a.wait_ns) {
             }
         }
         __syncthreads();
@@ -358,32 +534,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
-template <int D, int BK>
-cudaError_t launch_attn_t(const AttnArgs &a, const AttnMaps &maps, cudaStream_t stream) {
-    const size_t smem = (1 + kKStages + kVStages) * (size_t)(128 * D * 2) + 128 * 128 * 2 + 1024;
-    cudaError_t e = cudaFuncSetAttribute(gather_attn_kernel<D, BK>,
+template <int D, int BK, bool KF>
+cudaError_t launch_attn_t(const AttnArgs &a, const AttnMaps &maps, int num_sms, cudaStream_t stream) {
+    const size_t smem = AttnCfg<D>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(gather_attn_kernel<D, BK, KF>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    gather_attn_kernel<D, BK><<<(unsigned)a.rows, kAttnThreads, smem, stream>>>(maps, a);
+    const int grid = (int)(a.pairs < num_sms ? a.pairs : num_sms);
+    gather_attn_kernel<D, BK, KF><<<grid, kAttnThreads, smem, stream>>>(maps, a);
     return cudaGetLastError();
 }
 
+template <int D, int BK>
+cudaError_t launch_attn_k(const AttnArgs &a, const AttnMaps &maps, int num_sms, cudaStream_t stream) {
+    return a.k_fold ? launch_attn_t<D, BK, true>(a, maps, num_sms, stream)
+                    : launch_attn_t<D, BK, false>(a, maps, num_sms, stream);
+}
+
 template <int D>
-cudaError_t launch_attn_d(const AttnArgs &a, const AttnMaps &maps, cudaStream_t stream) {
+cudaError_t launch_attn_d(const AttnArgs &a, const AttnMaps &maps, int num_sms, cudaStream_t stream) {
     switch (a.Bk) {
-        case 16: return launch_attn_t<D, 16>(a, maps, stream);
-        case 32: return launch_attn_t<D, 32>(a, maps, stream);
-        case 64: return launch_attn_t<D, 64>(a, maps, stream);
-        case 128: return launch_attn_t<D, 128>(a, maps, stream);
+        case 16: return launch_attn_k<D, 16>(a, maps, num_sms, stream);
+        case 32: return launch_attn_k<D, 32>(a, maps, num_sms, stream);
+        case 64: return launch_attn_k<D, 64>(a, maps, num_sms, stream);
+        case 128: return launch_attn_k<D, 128>(a, maps, num_sms, stream);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_attention(const AttnArgs &a, const AttnMaps &maps, int, cudaStream_t stream) {
-    if (a.rows < 1) return cudaSuccess;
-    return a.D == 128 ? launch_attn_d<128>(a, maps, stream) : launch_attn_d<64>(a, maps, stream);
+cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t stream) {
+    if (a.pairs < 1) return cudaSuccess;
+    const size_t smem = sizeof(uint32_t) * 3 * (size_t)((a.nK + 31) / 32);
+    int64_t grid = a.pairs;
+    if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
+    pair_union_kernel<<<(unsigned)grid, kUnionThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnArgs &a, const AttnMaps &maps, int num_sms,
+                             cudaStream_t stream) {
+    if (a.pairs < 1) return cudaSuccess;
+    return a.D == 128 ? launch_attn_d<128>(a, maps, num_sms, stream)
+                      : launch_attn_d<64>(a, maps, num_sms, stream);
 }
 
 }  // namespace abatt

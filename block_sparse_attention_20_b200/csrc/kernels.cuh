@@ -70,20 +70,51 @@ size_t sample_smem_bytes(int nK);
 cudaError_t launch_sample(const SampleArgs &a, int num_sms, cudaStream_t stream);
 
 // ---- gather attention -----------------------------------------------------
-struct AttnArgs {
-    int64_t rows;  // query blocks
-    int nQ, N, D, Bk, nK;
-    int capacity;
-    float scale_log2;  // scale * log2(e)
+// Query blocks are processed in pairs of neighbours of the same head: pair
+// (h, j) holds blocks 2j and 2j+1 of head h (the last pair of a head is a
+// single block when nQ is odd).  A pre-pass merges the pair's two ascending
+// lists into one ascending union; every union block is gathered once and
+// used by both rows, each row masking the blocks it did not draw.
+__host__ __device__ __forceinline__ int64_t pairs_per_head(int nQ) { return (nQ + 1) / 2; }
+
+// Rows of pair `pr`: first row, and the second row or -1.
+__host__ __device__ __forceinline__ void pair_rows(int64_t pr, int nQ, int64_t *r0, int64_t *r1) {
+    const int64_t pph = pairs_per_head(nQ);
+    const int64_t h = pr / pph, j = pr - h * pph;
+    *r0 = h * nQ + 2 * j;
+    *r1 = (2 * j + 1 < nQ) ? *r0 + 1 : -1;
+}
+
+struct PairArgs {
+    int64_t rows, pairs;
+    int nQ, nK, capacity, cap_u;
     const int32_t *counts, *idx;
     const float *logw;
+    int32_t *ulen;  // [pairs]
+    int32_t *ublk;  // [pairs][cap_u]   ascending union of the two lists
+    float *ulw;     // [pairs][2][cap_u] log-weight of each row, -1 = not drawn
+    uint32_t *status;
+};
+cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t stream);
+
+struct AttnArgs {
+    int64_t rows, pairs;  // query blocks, row pairs
+    int nQ, N, D, Bk, nK;
+    int cap_u;
+    int k_fold;        // K tiles via head-folded 4-D boxes (needs N % 8 == 0)
+    float scale_log2;  // scale * log2(e)
+    const int32_t *ulen, *ublk;
+    const float *ulw;
     __nv_bfloat16 *O;  // [B*H][N][D]
     float *lse;        // optional [B*H][N]
     WsHeader *hdr;
     uint64_t wait_ns;
 };
 struct AttnMaps {
-    CUtensorMap q, k, v;
+    CUtensorMap q;  // [heads][N][D], box (64, 128, 1)
+    CUtensorMap k;  // k_fold: (64, 8 rows, 2 chunks, heads*N/8 groups), box (64, 8, 2, Bk/8)
+                    // else:   [heads][N][D], box (64, Bk, 1)
+    CUtensorMap v;  // (64, N rows, 2 chunks, heads), box (64, Bk, 2, 1)
 };
 cudaError_t launch_attention(const AttnArgs &a, const AttnMaps &maps, int num_sms,
                              cudaStream_t stream);

@@ -88,8 +88,8 @@ typedef enum abatt_call {
 } abatt_call;
 
 /* Bytes of device workspace `call` needs for this shape/config (256-byte
- * aligned base).  `capacity` is the list capacity used by ATTENTION
- * (ignored otherwise).  Host-only, no CUDA call. */
+ * aligned base; it does not depend on the list capacity).  Host-only, no
+ * CUDA call. */
 abatt_status abatt_workspace_size(abatt_call call, const abatt_shape *shape,
                                   const abatt_config *cfg, size_t *bytes);
 
@@ -127,10 +127,13 @@ abatt_status abatt_sample(const float *p, const abatt_shape *shape, const abatt_
  * softmax attention over the keys of its listed blocks only, each logit of
  * block b shifted by logw_b:
  *   O[q] = sum_t e^{l_t} v_t / sum_t e^{l_t},  l_t = s q.k_t + logw_{b(t)}.
- * Blocks are gathered from K/V into 128-key tensor-core tiles.  An empty
- * list gives O = 0 (and lse = -inf).  lse (optional, NULL to skip): fp32
+ * Each row's list must be strictly ascending (as abatt_sample writes it).
+ * Blocks are gathered from K/V into 128-key tensor-core tiles; two
+ * neighbouring query blocks (rows 2p, 2p+1) share the gathers of the union
+ * of their lists, each masking the blocks it did not draw.  An empty list
+ * gives O = 0 (and lse = -inf).  lse (optional, NULL to skip): fp32
  * [B][H][N], natural-log sum of exponentials per query.  Indices outside
- * [0, nK) are skipped and flagged ABATT_DEVFLAG_BADLIST. */
+ * [0, nK) or out of order are skipped and flagged ABATT_DEVFLAG_BADLIST. */
 abatt_status abatt_attention(const void *Q, const void *K, const void *V,
                              const abatt_shape *shape, const abatt_config *cfg,
                              const int32_t *counts, const int32_t *idx, const float *logw,

@@ -47,11 +47,14 @@ def test_workspace_sizes():
     B, H, N, d = 1, 40, 75600, 128
     fwd = _ws((B, H, N, d), cfg)
     sel = _ws((B, H, N, d), cfg, abatt.CALL_SELECT)
+    att = _ws((B, H, N, d), cfg, abatt.CALL_ATTENTION)
     assert _ws((B, H, N, d), cfg, abatt.CALL_SAMPLE) == 256
-    assert _ws((B, H, N, d), cfg, abatt.CALL_ATTENTION) == 256
     rows, nK = 40 * 591, 4725
-    # forward holds the selector's scratch plus p and capacity-nK lists
-    assert fwd >= sel + rows * nK * 12 + rows * 4
+    pairs = 40 * 296  # neighbouring query blocks of a head, 591 per head
+    # attention: per pair the union list (block, two log-weights) of at most nK blocks
+    assert att >= 256 + pairs * nK * 12
+    # forward holds the selector's and attention's scratch plus p and capacity-nK lists
+    assert fwd >= sel + (att - 256) + rows * nK * 12 + rows * 4
     assert fwd < 8 * 2**30
 
 

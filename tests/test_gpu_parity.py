@@ -171,6 +171,16 @@ def test_attention_ragged_shapes(d, Bk):
     _attn_check(Q, K, V, shape, Bk, rows, c, i, lw)
 
 
+@pytest.mark.parametrize("d,Bk", [(128, 16), (64, 32), (128, 128)])
+def test_attention_odd_blocks_per_head(d, Bk):
+    # nQ = 3 per head: the last query block of each head has no partner;
+    # N % 8 != 0 exercises the K gather that does not fold heads.
+    shape = (1, 3, 300, d)
+    Q, K, V = (synth.random_bf16(shape, s) for s in (13, 14, 15))
+    rows, c, i, lw = _random_lists(shape, Bk, 3000, 41 + Bk)
+    _attn_check(Q, K, V, shape, Bk, rows, c, i, lw)
+
+
 def test_attention_tiny_oracle_lists():
     w = synth.TINY
     Q, K, V = synth.generate(w)
@@ -214,7 +224,8 @@ def test_attention_empty_rows_and_bad_index():
     i2 = i.copy()
     i2[1, 0] = 10**6
     cfg = abatt.Config(kv_block=16)
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_ATTENTION, shape, cfg), dtype=torch.uint8,
+                     device="cuda")
     O = abatt.attention(Q.cuda(), K.cuda(), V.cuda(), torch.from_numpy(c).cuda(),
                         torch.from_numpy(i2).cuda(), torch.from_numpy(lw).cuda(), cfg,
                         workspace=ws)
