@@ -26,7 +26,7 @@ DEVFLAG_CAPACITY, DEVFLAG_TIMEOUT, DEVFLAG_BADLIST = 0x1, 0x2, 0x4
 EXPORTS = (
     "abatt_workspace_size", "abatt_select", "abatt_sample", "abatt_attention", "abatt_forward",
     "abatt_forward_intermediates", "abatt_read_status", "abatt_clear_status",
-    "abatt_status_string", "abatt_version",
+    "abatt_status_string", "abatt_version", "abatt_attention_noalloc",
 )
 
 
@@ -86,6 +86,7 @@ def lib():
         L.abatt_sample.argtypes = [P, S, C, P, P, P, i32, P, sz, P]
         L.abatt_attention.argtypes = [P, P, P, S, C, P, P, P, i32, P, P, P, sz, P]
         L.abatt_forward.argtypes = [P, P, P, S, C, P, P, P, sz, P]
+        L.abatt_attention_noalloc.argtypes = [P, P, P, S, C, P, P, P, i32, P, P, P, P]
         L.abatt_forward_intermediates.argtypes = [P, S, C, ctypes.POINTER(P), ctypes.POINTER(P),
                                                   ctypes.POINTER(P), ctypes.POINTER(P)]
         L.abatt_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
@@ -219,6 +220,27 @@ def attention(q, k, v, counts, idx, logw, cfg: Config, *, out=None, want_lse=Fal
                                  cap, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "abatt_attention")
     return (out, lse) if want_lse else out
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def attention_noalloc(q, k, v, counts, idx, logw, cfg: Config, *, out, lse=None, dev_status=None,
+                      stream=None):
+    """Gather attention through the entry point that allocates nothing.
+
+    For callers that cannot allocate device memory: its scratch is a fixed
+    64 MiB array inside the library, shared by every call on a device (calls
+    that overlap on the GPU race on it).  The caller supplies every input and
+    output buffer, including `out` (and `lse`, `dev_status` if wanted)."""
+    _check_bf16(q, k, v)
+    sh = _shape_of(q)
+    _check(lib().abatt_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(sh),
+                                         ctypes.byref(cfg._c(sh.d)), _ptr(counts), _ptr(idx),
+                                         _ptr(logw), idx.shape[1], _ptr(out), _ptr(lse),
+                                         _ptr(dev_status), _stream(stream)),
+           "abatt_attention_noalloc")
+    return out
 
 
 def forward(q, k, v, cfg: Config, *, out=None, want_lse=False, workspace=None, stream=None):

@@ -263,6 +263,29 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     return cuda_status(launch_attention(a, m, sms, st));
 }
 
+// Scratch of abatt_attention_noalloc: status word and pair unions, in the
+// library's device image (no allocation at call time).  Device code could
+// name it directly; host code needs its address from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ABATT_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device, looked up once
+// per device with that device current.
+abatt_status noalloc_scratch(void **ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ABATT_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ABATT_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return ABATT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -349,6 +372,35 @@ abatt_status abatt_attention(const void *Q, const void *K, const void *V,
     if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
     return run_attention(Q, K, V, g, cfg, counts, idx, logw, capacity, O, lse, workspace, L, sms,
                          st);
+}
+
+abatt_status abatt_attention_noalloc(const void *Q, const void *K, const void *V,
+                                     const abatt_shape *shape, const abatt_config *cfg,
+                                     const int32_t *counts, const int32_t *idx, const float *logw,
+                                     int capacity, void *O, float *lse, uint32_t *dev_status,
+                                     void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!Q || !K || !V || !O || !counts || !idx || !logw || capacity < 1)
+        return ABATT_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+        return ABATT_ERR_ALIGNMENT;
+    const Layout L = layout(ABATT_CALL_ATTENTION, g);
+    if (L.total > (size_t)ABATT_NOALLOC_SCRATCH_BYTES) return ABATT_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the status word must start at zero; the union lists are fully rewritten
+    if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
+    s = run_attention(Q, K, V, g, cfg, counts, idx, logw, capacity, O, lse, scratch, L, sms, st);
+    if (s != ABATT_OK) return s;
+    if (dev_status && cudaMemcpyAsync(dev_status, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice,
+                                      st) != cudaSuccess)
+        return ABATT_ERR_CUDA;
+    return ABATT_OK;
 }
 
 abatt_status abatt_forward(const void *Q, const void *K, const void *V,

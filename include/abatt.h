@@ -153,6 +153,37 @@ abatt_status abatt_forward_intermediates(void *workspace, const abatt_shape *sha
                                          const abatt_config *cfg, float **p, int32_t **counts,
                                          int32_t **idx, float **logw);
 
+/* Gather attention without a workspace, for callers that cannot allocate
+ * device memory: for example code running inside a memory pool or arena it
+ * does not own, a plugin whose host application forbids allocation during
+ * inference, or a process that must not trigger allocation (and its
+ * synchronisation) on a latency-critical path.  No counterpart in the paper:
+ * this is an interface convenience of this library.
+ *
+ * Computes exactly what abatt_attention computes, with the same arguments
+ * except the workspace.  Its scratch (status word and the per-pair union
+ * lists) lives in a fixed array of ABATT_NOALLOC_SCRATCH_BYTES inside the
+ * library's device image; every GPU that loads the library holds that
+ * array until the process exits.  Shapes whose scratch would exceed it are
+ * rejected with ABATT_ERR_UNSUPPORTED before any launch (the scratch needed
+ * is abatt_workspace_size(ABATT_CALL_ATTENTION, ...)).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Every
+ * call on a device shares the one array and leaves its contents behind:
+ * calls that may overlap on the GPU (different streams without ordering, or
+ * concurrent host threads) race on it and must be serialised by the caller.
+ * The call allocates and frees nothing.
+ *
+ * dev_status (device pointer, NULL to skip) receives the ABATT_DEVFLAG_*
+ * bits of this call, asynchronously on `stream`. */
+#define ABATT_NOALLOC_SCRATCH_BYTES (64u << 20)
+abatt_status abatt_attention_noalloc(const void *Q, const void *K, const void *V,
+                                     const abatt_shape *shape, const abatt_config *cfg,
+                                     const int32_t *counts, const int32_t *idx, const float *logw,
+                                     int capacity, void *O, float *lse, uint32_t *dev_status,
+                                     void *stream);
+
 /* Synchronously copy the device status word at the start of `workspace` to
  * *flags (ABATT_DEVFLAG_* bits) after `stream` drains.  Returns
  * ABATT_ERR_DEVICE if any bit is set, ABATT_OK otherwise. */

@@ -1,0 +1,73 @@
+"""The allocation-free attention entry point (abatt_attention_noalloc).
+
+Some callers cannot allocate device memory at call time (they run inside a
+memory pool they do not own, or their host forbids allocation on the
+inference path).  For them the library offers one attention call whose
+scratch lives in a fixed array inside the library.  These checks call it
+through the C ABI and compare it with the regular abatt_attention on the same
+inputs, twice in a row (the second call reuses the scratch the first left
+behind), and check that oversized problems are refused before any launch.
+
+This file is collected last on purpose, and passes both alone and after the
+other GPU tests.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_20_b200 import abatt, synth
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 5e-3
+MAX_ABS = 2e-2
+
+
+def _lists(shape, Bk, bp, seed):
+    B, H, N, d = shape
+    nK = -(-N // Bk)
+    rows = np.arange(B * H * (-(-N // 128)))
+    p = synth.random_probs(len(rows), nK, seed, 0.3)
+    c, i, lw, _, _ = oracle.sample(p, shape, rows, bp, seed, Bk=Bk)
+    return (torch.from_numpy(c).cuda(), torch.from_numpy(i).cuda(), torch.from_numpy(lw).cuda())
+
+
+def _close(a, b):
+    a = a.float().cpu().numpy()
+    b = b.float().cpu().numpy()
+    rel = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+    return rel <= REL_L2 and np.max(np.abs(a - b)) <= MAX_ABS
+
+
+@pytest.mark.parametrize("shape,Bk", [((1, 2, 4096, 64), 16), ((2, 3, 1000, 128), 32)])
+def test_noalloc_matches_attention_twice(shape, Bk):
+    Q, K, V = (synth.random_bf16(shape, s).cuda() for s in (91, 92, 93))
+    counts, idx, logw = _lists(shape, Bk, 1500, 94)
+    cfg = abatt.Config(kv_block=Bk)
+    ref, ref_lse = abatt.attention(Q, K, V, counts, idx, logw, cfg, want_lse=True)
+    status = torch.full((1,), 0xFFFF, dtype=torch.int32, device="cuda")
+    for _ in range(2):
+        out = torch.full_like(Q, float("nan"))
+        lse = torch.full(shape[:3], float("nan"), dtype=torch.float32, device="cuda")
+        abatt.attention_noalloc(Q, K, V, counts, idx, logw, cfg, out=out, lse=lse, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert _close(out, ref)
+        fin = torch.isfinite(ref_lse)
+        assert torch.equal(fin, torch.isfinite(lse))
+        assert torch.max(torch.abs(lse[fin] - ref_lse[fin])).item() <= 1e-2
+
+
+def test_noalloc_refuses_shapes_beyond_its_scratch():
+    cfg = abatt.Config(kv_block=16)
+    big = (1, 40, 75600, 128)  # needs far more than the fixed scratch
+    assert abatt.workspace_size(abatt.CALL_ATTENTION, big, cfg) > abatt.NOALLOC_SCRATCH_BYTES
+    sh = abatt._Shape(*big)
+    one = torch.zeros(1, dtype=torch.int32, device="cuda")  # never read: refused on the host
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    code = abatt.lib().abatt_attention_noalloc(
+        abatt._ptr(x), abatt._ptr(x), abatt._ptr(x), abatt.ctypes.byref(sh),
+        abatt.ctypes.byref(cfg._c(128)), abatt._ptr(one), abatt._ptr(one), abatt._ptr(one), 1,
+        abatt._ptr(x), None, None, None)
+    assert code == 2  # ABATT_ERR_UNSUPPORTED
