@@ -3,12 +3,17 @@
 // Attention", abstract, selector sentence: queries are clustered only within
 // each query block, without permuting tokens).
 //
-// One CTA of 128 threads per query block; thread r owns query row r.  The
-// block's queries sit in shared memory as fp32, transposed with a padded
-// stride so both the per-row distance loop and the per-dimension centroid
-// sums read conflict-free.  Rounds are deterministic: the centroid update
-// sums each cluster's rows in ascending row order (a stable counting sort by
-// cluster, built from warp ballots).
+// One CTA of 128 threads (4 warps) per query block.  The block's queries stay
+// in shared memory as bf16 (exact copies of the inputs).  Per round:
+//   - distances: ||c_j||^2 - 2 q.c_j, the dot products on the tensor cores
+//     (mma.sync m16n8k16, bf16 in, fp32 accumulate) with each fp32 centroid
+//     split into a bf16 high part and a bf16 residual, so the products carry
+//     about 16 significant bits of the centroid; warp w takes rows
+//     32w..32w+31; the argmin (ties to the lower index) is reduced across the
+//     four lanes that share a row;
+//   - update: a stable counting sort of the rows by cluster (warp ballots),
+//     then thread x sums dimension x of each cluster's rows in ascending row
+//     order (deterministic), centroid = sum / size.
 //
 // Rules (open in the abstract, fixed here): C_eff = min(C, n) clusters;
 // centroid j starts at row floor(j*n/C_eff); squared Euclidean distance,
@@ -28,12 +33,24 @@ namespace {
 constexpr int kKmThreads = 128;
 constexpr int kMaxC = 16;
 
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a) {
-    constexpr int LD = 129;  // padded row stride of the transposed block
-    extern __shared__ __align__(16) float km_smem[];
-    float *qT = km_smem;                     // [D][LD]
-    float *cent = qT + D * LD;               // [kMaxC][D]
+    constexpr int LDQ = D + 8;  // bf16 row stride: 4*row + column-pair spreads the banks
+    extern __shared__ __align__(16) unsigned char km_smem[];
+    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(km_smem);             // [128][LDQ]
+    float *cent = reinterpret_cast<float *>(km_smem + 128 * LDQ * 2);            // [kMaxC][D]
+    __nv_bfloat16 *chi = reinterpret_cast<__nv_bfloat16 *>(cent + kMaxC * D);    // [kMaxC][LDQ]
+    __nv_bfloat16 *clo = chi + kMaxC * LDQ;                                      // [kMaxC][LDQ]
+    __shared__ float cnorm[kMaxC];
     __shared__ int assign_s[128];
     __shared__ int order_s[128];
     __shared__ uint32_t mask_s[4][kMaxC];
@@ -42,7 +59,12 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
     __shared__ int woff_s[4][kMaxC];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, cq = lane & 3;  // mma fragment coordinates
     const int C = a.C;
+    const uint32_t *qw = reinterpret_cast<const uint32_t *>(qs);
+    const uint32_t *hw = reinterpret_cast<const uint32_t *>(chi);
+    const uint32_t *lw = reinterpret_cast<const uint32_t *>(clo);
+    constexpr int LDW = LDQ / 2;  // row stride in 32-bit words
 
     for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
         const int i = (int)(row % a.nQ);
@@ -51,53 +73,91 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         const int ce = min(C, n);
         const __nv_bfloat16 *qblk = a.Q + (bh * (int64_t)a.N + (int64_t)i * 128) * D;
 
-        // load the block (thread r <- row r), transposed into qT[x][r]
-        if (tid < n) {
+        // the block's queries, row r by thread r; missing rows are zero
+        {
             const uint4 *src = reinterpret_cast<const uint4 *>(qblk + (int64_t)tid * D);
+            uint4 *dst = reinterpret_cast<uint4 *>(qs + tid * LDQ);
 #pragma unroll 4
-            for (int v = 0; v < D / 8; ++v) {
-                uint4 u = src[v];
-                const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&u);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) qT[(v * 8 + k) * LD + tid] = __bfloat162float(e[k]);
-            }
+            for (int v = 0; v < D / 8; ++v) dst[v] = tid < n ? src[v] : make_uint4(0, 0, 0, 0);
         }
         __syncthreads();
         for (int e = tid; e < kMaxC * D; e += kKmThreads) {
             const int j = e / D, x = e % D;
-            cent[e] = j < ce ? qT[x * LD + (int)(((int64_t)j * n) / ce)] : 0.0f;
+            cent[e] = j < ce ? __bfloat162float(qs[(int)(((int64_t)j * n) / ce) * LDQ + x]) : 0.0f;
         }
         __syncthreads();
 
         const int rounds = a.iters > 0 ? a.iters : 1;
         for (int it = 0; it < rounds; ++it) {
-            // ---- assignment ----
-            int best = -1;
-            if (tid < n) {
-                float acc[kMaxC];
+            // ---- centroid operands: bf16 hi + lo, squared norms ----
+            for (int e = tid; e < kMaxC * D; e += kKmThreads) {
+                const int j = e / D, x = e % D;
+                const float c = cent[e];
+                const __nv_bfloat16 h = __float2bfloat16_rn(c);
+                chi[j * LDQ + x] = h;
+                clo[j * LDQ + x] = __float2bfloat16_rn(c - __bfloat162float(h));
+            }
+            if (tid < kMaxC) {
+                float s = 0.0f;
+                for (int x = 0; x < D; ++x) s = fmaf(cent[tid * D + x], cent[tid * D + x], s);
+                cnorm[tid] = s;
+            }
+            __syncthreads();
+
+            // ---- assignment: q.c on tensor cores, argmin over centroids ----
+            const int nt = (ce + 7) >> 3;  // 8-wide centroid tiles
+            float bestd[2][2];
+            int besti[2][2];
 #pragma unroll
-                for (int j = 0; j < kMaxC; ++j) acc[j] = 0.0f;
-#pragma unroll 4
-                for (int x = 0; x < D; ++x) {
-                    const float q = qT[x * LD + tid];
+            for (int m = 0; m < 2; ++m) {
+                const int r0 = warp * 32 + m * 16;
 #pragma unroll
-                    for (int j = 0; j < kMaxC; ++j) {
-                        if (j < ce) {
-                            const float df = q - cent[j * D + x];
-                            acc[j] = fmaf(df, df, acc[j]);
+                for (int h = 0; h < 2; ++h) { bestd[m][h] = __int_as_float(0x7f800000); besti[m][h] = 0; }
+                for (int t = 0; t < nt; ++t) {
+                    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                    for (int k0 = 0; k0 < D; k0 += 16) {
+                        const int kw = (k0 >> 1) + cq;  // word of column pair k0 + 2cq
+                        uint32_t af[4];
+                        af[0] = qw[(r0 + g) * LDW + kw];
+                        af[1] = qw[(r0 + g + 8) * LDW + kw];
+                        af[2] = qw[(r0 + g) * LDW + kw + 4];
+                        af[3] = qw[(r0 + g + 8) * LDW + kw + 4];
+                        const int cj = t * 8 + g;
+                        mma_bf16_16816(acc, af, hw[cj * LDW + kw], hw[cj * LDW + kw + 4]);
+                        mma_bf16_16816(acc, af, lw[cj * LDW + kw], lw[cj * LDW + kw + 4]);
+                    }
+                    // acc[0..1]: row g, centroids t*8+2cq+{0,1}; acc[2..3]: row g+8
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int j = t * 8 + 2 * cq + u;
+                            const float dj = j < ce ? fmaf(-2.0f, acc[2 * h + u], cnorm[j])
+                                                    : __int_as_float(0x7f800000);
+                            if (dj < bestd[m][h]) { bestd[m][h] = dj; besti[m][h] = j; }
+                        }
+                }
+                // combine the four lanes of each row (ties to the lower index)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int o = 1; o < 4; o <<= 1) {
+                        const float od = __shfl_xor_sync(0xffffffffu, bestd[m][h], o);
+                        const int oi = __shfl_xor_sync(0xffffffffu, besti[m][h], o);
+                        if (od < bestd[m][h] || (od == bestd[m][h] && oi < besti[m][h])) {
+                            bestd[m][h] = od;
+                            besti[m][h] = oi;
                         }
                     }
+                if (cq == 0) {
+                    assign_s[r0 + g] = (r0 + g) < n ? besti[m][0] : -1;
+                    assign_s[r0 + g + 8] = (r0 + g + 8) < n ? besti[m][1] : -1;
                 }
-                float bd = acc[0];
-                best = 0;
-#pragma unroll
-                for (int j = 1; j < kMaxC; ++j)
-                    if (j < ce && acc[j] < bd) {
-                        bd = acc[j];
-                        best = j;
-                    }
             }
-            assign_s[tid] = best;
+            __syncthreads();
+            const int best = assign_s[tid];
+
             // ---- stable counting sort of rows by cluster ----
             for (int j = 0; j < ce; ++j) {
                 const uint32_t m = __ballot_sync(0xffffffffu, best == j);
@@ -130,7 +190,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                     if (c == 0) continue;
                     float s = 0.0f;
                     const int b0 = base_s[j];
-                    for (int e = 0; e < c; ++e) s += qT[x * LD + order_s[b0 + e]];
+                    for (int e = 0; e < c; ++e) s += __bfloat162float(qs[order_s[b0 + e] * LDQ + x]);
                     cent[j * D + x] = s / (float)c;
                 }
             }
@@ -161,7 +221,10 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
 
 }  // namespace
 
-size_t kmeans_smem_bytes(int D) { return sizeof(float) * (size_t)(D * 129 + kMaxC * D); }
+size_t kmeans_smem_bytes(int D) {
+    const int ldq = D + 8;
+    return (size_t)128 * ldq * 2 + sizeof(float) * kMaxC * D + 2 * (size_t)kMaxC * ldq * 2;
+}
 
 cudaError_t launch_kmeans(const KmeansArgs &a, int num_sms, cudaStream_t stream) {
     int64_t grid = a.rows;
