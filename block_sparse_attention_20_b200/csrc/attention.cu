@@ -19,24 +19,28 @@
 //
 //   tensor core, per tile t:   S0(t)  PV1(t-1)  S1(t)  PV0(t)
 //
-// Warp roles (384 threads):
+// Warp roles (576 threads):
 //   warp 0      TMA producer: Q of both rows, then K(t), V(t) into a ring;
 //   warp 1      tensor-memory owner and tcgen05 MMA issuer:
 //               S_s = Q_s K^T (fp32, 128 TMEM columns per row),
 //               O_s += P_s V  (P_s read back from the columns S_s used);
-//   warps 2-3   idle;
-//   warps 4-7   softmax of row 0, warps 8-11 softmax of row 1 (thread = query):
-//               one TMEM read of the tile, raw per-block maxima, tile maximum
-//               of s*log2(e)*S + log-weight (base 2), lazy running maximum
-//               (O is rescaled only when it grows by more than 8), P in bf16
-//               back into tensor memory chunk by chunk, final O / l to bf16.
+//   warps 2-17  softmax, four warpgroups: row s of the pair and column half
+//               hh of each tile per warpgroup (thread = query): raw per-block
+//               maxima of its 64 columns, the two halves' tile maxima of
+//               s*log2(e)*S + log-weight (base 2) exchanged through shared
+//               memory, lazy running maximum (O is rescaled only when it grows
+//               by more than 8), P in bf16 back into tensor memory, final
+//               O / l to bf16 (each half writes its 64 output columns).
+//               The softmax latency of a tile sits on each row's critical
+//               path (P replaces S in tensor memory, so S(t+1) waits for
+//               PV(t)); splitting the columns halves it.
 #include "kernels.cuh"
 
 namespace abatt {
 
 namespace {
 
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 576;
 #define kNegInf (-__int_as_float(0x7f800000))
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -147,7 +151,7 @@ template <int D>
 struct AttnCfg {
     static constexpr int CH = D / 64;
     static constexpr uint32_t TILE = 128u * D * 2u;
-    static constexpr int ST = D == 128 ? 5 : 10;  // K/V ring stages
+    static constexpr int ST = D == 128 ? 4 : 9;  // K/V ring stages
     static constexpr size_t SMEM = (size_t)(2 + ST) * TILE + 1024;
 };
 
@@ -173,6 +177,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __shared__ __align__(8) uint64_t bar_drain;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
+    __shared__ float xchg[2][2][2][128];  // [row s][tile parity][column half][query]
+    __shared__ float xsum[2][2][128];      // [row s][column half][query] row sums
+    __shared__ __align__(8) uint64_t bar_x[2];  // the two halves of row s have exchanged
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT))
@@ -185,15 +192,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&bar_qf[s], 1);
             mbar_init(&bar_qe[s], 1);
             mbar_init(&bar_sf[s], 1);
-            mbar_init(&bar_pf[s], 4);
+            mbar_init(&bar_pf[s], 8);
             mbar_init(&bar_of[s], 1);
-            mbar_init(&bar_oe[s], 4);
+            mbar_init(&bar_oe[s], 8);
         }
         for (int s = 0; s < ST; ++s) {
             mbar_init(&bar_kvf[s], 1);
             mbar_init(&bar_kve[s], 1);
         }
         mbar_init(&bar_drain, 1);
+        mbar_init(&bar_x[0], 8);
+        mbar_init(&bar_x[1], 8);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -354,15 +363,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 rp = base + 2 * n;
             }
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
         // ================================ softmax =====================================
-        const int s = (warp - 4) >> 2;  // row of the pair
-        const int wq = warp & 3;        // tensor-memory lane quarter
-        const int r = wq * 32 + lane;   // query row within the block == TMEM lane
+        constexpr int HB = BPT >= 2 ? BPT / 2 : 1;  // blocks (or block parts) per column half
+        const int sw = warp - 2;
+        const int s = sw >> 3;         // row of the pair
+        const int hh = (sw >> 2) & 1;  // column half of each tile
+        const int wq = warp & 3;       // tensor-memory lane quarter
+        const int r = wq * 32 + lane;  // query row within the block == TMEM lane
         const uint32_t t_lane = (uint32_t)(wq * 32) << 16;
         const uint32_t s_col = tmem + t_lane + s * 128;
         const uint32_t o_col = tmem + t_lane + 256 + s * 128;
-        uint32_t s_uses = 0, o_uses = 0;
+        uint32_t s_uses = 0, o_uses = 0, x_uses = 0;
+        // both halves of the row have published their values (bounded wait)
+        auto exchange = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_x[s]);
+            const bool got = mbar_wait(&bar_x[s], x_uses & 1, wc, 0x20b);
+            ++x_uses;
+            return got;
+        };
         bool ok = true;
         for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
             int64_t rr[2];
@@ -378,14 +398,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float *lw = a.ulw + (pr * 2 + s) * (int64_t)a.cap_u;
             float m_run = kNegInf, l = 0.0f;
             for (int t = 0; t < n; ++t) {
-                // per-block base-2 log-weight (-inf where this row did not draw
-                // the block or the slot is empty); the one block that can be
-                // cut by N is the last block of the sequence
-                float bias[BPT];
+                // this half's blocks: base-2 log-weight (-inf where this row did
+                // not draw the block or the slot is empty); the block that can
+                // be cut by N is the last block of the sequence
+                float bias[HB];
                 int tail_k = -1, tail_keep = BK;
 #pragma unroll
-                for (int k = 0; k < BPT; ++k) {
-                    const int j = t * BPT + k;
+                for (int k = 0; k < HB; ++k) {
+                    const int j = t * BPT + (BPT >= 2 ? hh * HB + k : 0);
                     bias[k] = kNegInf;
                     if (j < U) {
                         const float w = __ldg(lw + j);
@@ -401,63 +421,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(&bar_sf[s], s_uses & 1, wc, 0x208)) { ok = false; break; }
                 ++s_uses;
                 tc_fence_after();
-
-                uint32_t v[4][32];
+                uint32_t v[2][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, v[c]);
+                for (int c = 0; c < 2; ++c) tmem_ld32(s_col + hh * 64 + c * 32, v[c]);
                 tmem_wait_ld();
-                if (masked) {  // keys past N inside the last block of the sequence
+                // column (within the tile) of v[c][j]: 64*hh + 32*c + j; its block
+                // slot within this half: (32c + j) / BK (or 0 for blocks wider
+                // than a half); its key within the block: column % BK
+                if (masked) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if ((c * 32 + j) / BK == tail_k && (c * 32 + j) % BK >= tail_keep)
-                                v[c][j] = __float_as_uint(kNegInf);
+                        for (int j = 0; j < 32; ++j) {
+                            const int col = hh * 64 + c * 32 + j;
+                            const int k = BPT >= 2 ? (c * 32 + j) / BK : 0;
+                            if (k == tail_k && col % BK >= tail_keep) v[c][j] = __float_as_uint(kNegInf);
+                        }
                 }
-                float bmax[BPT];
+                float bmax[HB];
 #pragma unroll
-                for (int k = 0; k < BPT; ++k) bmax[k] = kNegInf;
+                for (int k = 0; k < HB; ++k) bmax[k] = kNegInf;
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int k = (c * 32 + j) / BK;
+                        const int k = BPT >= 2 ? (c * 32 + j) / BK : 0;
                         bmax[k] = fmaxf(bmax[k], __uint_as_float(v[c][j]));
                     }
-                float tmax = kNegInf;
+                float hmax = kNegInf;
 #pragma unroll
-                for (int k = 0; k < BPT; ++k) tmax = fmaxf(tmax, fmaf(bmax[k], a.scale_log2, bias[k]));
+                for (int k = 0; k < HB; ++k) hmax = fmaxf(hmax, fmaf(bmax[k], a.scale_log2, bias[k]));
+                // both halves' S reads are done once the exchange completes, so P
+                // may then overwrite S anywhere in the row's columns
+                xchg[s][t & 1][hh][r] = hmax;
+                tc_fence_before();
+                if (!exchange()) { ok = false; break; }
+                tc_fence_after();
+                const float tmax = fmaxf(hmax, xchg[s][t & 1][hh ^ 1][r]);
                 const bool need = tmax > m_run + kRescaleThreshold;
                 const float m_use = need ? tmax : m_run;
                 const float alpha = need ? ((m_run == kNegInf) ? 0.0f : ex2_approx(m_run - tmax)) : 1.0f;
                 const float m_sub = (m_use == kNegInf) ? 0.0f : m_use;
 #pragma unroll
-                for (int k = 0; k < BPT; ++k) bias[k] -= m_sub;  // now the exponent offset
+                for (int k = 0; k < HB; ++k) bias[k] -= m_sub;  // now the exponent offset
                 float rs = 0.0f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        const int k0 = (c * 32 + j) / BK, k1 = (c * 32 + j + 1) / BK;
+                        const int k0 = BPT >= 2 ? (c * 32 + j) / BK : 0;
+                        const int k1 = BPT >= 2 ? (c * 32 + j + 1) / BK : 0;
                         const float p0 = ex2_approx(fmaf(__uint_as_float(v[c][j]), a.scale_log2, bias[k0]));
                         const float p1 = ex2_approx(fmaf(__uint_as_float(v[c][j + 1]), a.scale_log2, bias[k1]));
                         rs += p0 + p1;
                         pk[j >> 1] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(s_col + c * 16, pk);
+                    tmem_st16(s_col + hh * 32 + c * 16, pk);
                 }
-                // rescale O (after P, so the scores are dead): the commit that
-                // signalled S(t) covers the previous PV of this row
+                // rescale this half's O columns (after P, so the scores are
+                // dead): the commit that signalled S(t) covers the previous PV
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = 0; c < D / 64; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(o_col + c * 32, o);
+                        const uint32_t oa = o_col + hh * (D / 2) + c * 32;
+                        tmem_ld32(oa, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st32(o_col + c * 32, o);
+                        tmem_st32(oa, o);
                     }
                 }
                 tmem_wait_st();
@@ -468,24 +501,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 m_run = m_use;
             }
             if (!ok) break;
-            __nv_bfloat16 *orow = a.O + tok * D;
+            __nv_bfloat16 *orow = a.O + tok * D + hh * (D / 2);
             if (n == 0) {  // no block at all: O = 0, lse = -inf
                 if (r < nrows) {
 #pragma unroll
-                    for (int q = 0; q < D / 8; ++q) reinterpret_cast<uint4 *>(orow)[q] = make_uint4(0, 0, 0, 0);
-                    if (a.lse) a.lse[tok] = kNegInf;
+                    for (int q = 0; q < D / 16; ++q) reinterpret_cast<uint4 *>(orow)[q] = make_uint4(0, 0, 0, 0);
+                    if (a.lse && hh == 0) a.lse[tok] = kNegInf;
                 }
                 continue;
             }
-            // epilogue: O / l -> bf16, then release O to this slot's next row
+            // epilogue: the row sum is split over the two halves
+            xsum[s][hh][r] = l;
+            if (!exchange()) { ok = false; break; }
+            l += xsum[s][hh ^ 1][r];
             if (!mbar_wait(&bar_of[s], o_uses & 1, wc, 0x209)) { ok = false; break; }
             ++o_uses;
             tc_fence_after();
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t o[32];
-                tmem_ld32(o_col + c * 32, o);
+                tmem_ld32(o_col + hh * (D / 2) + c * 32, o);
                 tmem_wait_ld();
                 if (r < nrows) {
 #pragma unroll
@@ -502,7 +538,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_oe[s]);
-            if (a.lse && r < nrows) a.lse[tok] = l > 0.0f ? (m_run + __log2f(l)) * kLn2 : kNegInf;
+            if (a.lse && hh == 0 && r < nrows) a.lse[tok] = l > 0.0f ? (m_run + __log2f(l)) * kLn2 : kNegInf;
         }
         tc_fence_before();
     }
