@@ -298,19 +298,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t rp = 0;  // ring position of K(t); V(t) is rp+1
             uint32_t q_uses[2] = {0, 0}, pv_ops[2] = {0, 0}, o_items[2] = {0, 0};
             bool ok = true;
-            const uint32_t q_addr0 = smem_u32(sQ), ring_addr = smem_u32(sRing);
+            const uint32_t q_addr0 = smem_u32(sQ), ring_addr = smem_u32(sRing);  // < 256 KB: the
+            // 14-bit address field of a descriptor never carries into the next field
             auto op_s = [&](int s, uint32_t kpos, bool release, bool last) -> bool {
                 const int stg = kpos % ST;
                 if (!mbar_wait(&bar_kvf[stg], (kpos / ST) & 1, wc, 0x203)) return false;
                 tc_fence_after();
-                const uint32_t qa = q_addr0 + s * TILE, ka = ring_addr + stg * TILE;
+                // descriptors built once per op; each k-step adds its byte offset / 16
+                const uint64_t qd = sdesc_sw128(q_addr0 + s * TILE, 16, 1024);
+                const uint64_t kd = sdesc_sw128(ring_addr + stg * TILE, 16, KFOLD ? CH * 1024 : 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
                     const uint32_t koff =
                         KFOLD ? (kk >> 2) * 1024 + (kk & 3) * 32 : (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_bf16_ss(tmem + s * 128, sdesc_sw128(qa + qoff, 16, 1024),
-                                 sdesc_sw128(ka + koff, 16, KFOLD ? CH * 1024 : 1024), idesc_s, kk > 0);
+                    umma_bf16_ss(tmem + s * 128, qd + (qoff >> 4), kd + (koff >> 4), idesc_s, kk > 0);
                 }
                 if (release) umma_commit(&bar_kve[stg]);
                 umma_commit(&bar_sf[s]);
@@ -325,12 +327,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int stg = vpos % ST;
                 if (!mbar_wait(&bar_kvf[stg], (vpos / ST) & 1, wc, 0x206)) return false;
                 tc_fence_after();
-                const uint32_t va = ring_addr + stg * TILE;
+                const uint64_t vd = sdesc_sw128(ring_addr + stg * TILE, BK * 128, 1024);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint32_t boff = (uint32_t)((16 * j) / BK) * BLK + (uint32_t)((16 * j) % BK) * 128;
-                    umma_bf16_ts(tmem + 256 + s * 128, tmem + s * 128 + j * 8,
-                                 sdesc_sw128(va + boff, BK * 128, 1024), idesc_o,
+                    umma_bf16_ts(tmem + 256 + s * 128, tmem + s * 128 + j * 8, vd + (boff >> 4), idesc_o,
                                  (t > 0 || j > 0) ? 1u : 0u);
                 }
                 if (release) umma_commit(&bar_kve[stg]);

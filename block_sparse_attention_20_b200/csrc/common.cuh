@@ -65,6 +65,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep until the phase completes or
+// `hint_ns` nanoseconds pass, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -86,9 +100,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        // sleep until the phase completes (or ~20 us pass): no issue slots
+        // are burnt polling while other warps of the SM do the work
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (*w.abort) return false;
-        if ((it & 63u) == 63u && globaltimer_ns() - t0 > w.limit_ns) {
+        if (globaltimer_ns() - t0 > w.limit_ns) {
             *w.abort = 1;
             if (w.hdr) {
                 atomicOr(&w.hdr->status, ABATT_DEVFLAG_TIMEOUT);
