@@ -4,11 +4,14 @@
 // sampling sentence: blocks are drawn in proportion to the estimates and
 // re-weighted by the inverse inclusion probability).
 //
-// One CTA per row (query block).  The row's probabilities stay in shared
-// memory; the water-filling rounds, the Philox draws and the ordered
-// compaction (warp ballot + block prefix sum) all run from there.  Every
-// decision is integer arithmetic on 48-bit fixed-point weights, so the
-// result does not depend on the launch configuration.
+// One CTA of 256 threads per row (query block).  The row's 48-bit
+// fixed-point weights are built once into shared memory; the water-filling
+// rounds, the Philox draws and the ordered compaction all run from there.
+// Thread t owns groups of four consecutive blocks (one Philox block yields
+// their four draws); positions in the list come from a block-wide scan of the
+// per-thread counts, so the list is ascending.  Every decision is integer
+// arithmetic on the fixed-point weights: the result does not depend on the
+// launch configuration.
 #include "kernels.cuh"
 
 namespace abatt {
@@ -17,13 +20,25 @@ namespace {
 
 constexpr int kSampleThreads = 256;
 constexpr int kSampleWarps = kSampleThreads / 32;
+constexpr int kCacheMaxBlocks = 8192;  // weights cached in shared memory up to this nK
 
+// round-half-even(p * 2^48) for p clamped to [0, 1] (NaN and negatives -> 0),
+// from the float's exponent and mantissa with integer shifts only.
 __device__ __forceinline__ int64_t to_fixed48(float p) {
-    // p * 2^48 is exact in fp32 (a power-of-two scaling of a value in [0, 1]);
-    // the conversion rounds half to even.
-    if (!(p > 0.0f)) return 0;  // zero, negative, NaN
-    if (p > 1.0f) p = 1.0f;
-    return __float2ll_rn(p * 281474976710656.0f);
+    if (!(p > 0.0f)) return 0;
+    if (p >= 1.0f) return int64_t(1) << 48;
+    const uint32_t bits = __float_as_uint(p);
+    const int e = (int)(bits >> 23);                      // biased exponent, 0 for subnormals
+    const uint32_t m = (bits & 0x7fffffu) | (e ? 0x800000u : 0u);
+    // value = m * 2^(e' - 150) * 2^48 with e' = max(e, 1) (subnormals use 1)
+    const int sh = (e ? e : 1) - 150 + 48;                // left shift of m (negative: right)
+    if (sh >= 0) return (int64_t)m << sh;                 // exact, < 2^48 since p < 1
+    const int rs = -sh;
+    if (rs > 24) return 0;                                // m < 2^24 <= 2^(rs-1): below one half
+    const uint32_t q = m >> rs;
+    const uint32_t rem = m & ((1u << rs) - 1u);
+    const uint32_t half = 1u << (rs - 1);
+    return (int64_t)(q + ((rem > half || (rem == half && (q & 1u))) ? 1u : 0u));
 }
 
 // Philox4x32-10 (Salmon et al., SC 2011): ten rounds, published multipliers
@@ -63,22 +78,39 @@ __device__ __forceinline__ bool draw_below(uint32_t U, uint64_t T, uint64_t RP) 
     return lhs_hi < rhs_hi || (lhs_hi == rhs_hi && lhs_lo < rhs_lo);
 }
 
-__global__ void __launch_bounds__(kSampleThreads)
-    sample_compact_kernel(SampleArgs a) {
+template <bool CACHED>
+__global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    float *ps = reinterpret_cast<float *>(smem_raw);                         // [nK]
-    uint8_t *sat = reinterpret_cast<uint8_t *>(smem_raw + sizeof(float) * a.nK_pad);  // [nK]
+    // CACHED: int64 weights [nK_pad]; else fp32 p [nK_pad].  Then sat bytes [nK_pad].
+    int64_t *Pw = reinterpret_cast<int64_t *>(smem_raw);
+    float *ps = reinterpret_cast<float *>(smem_raw);
+    uint8_t *sat = smem_raw + (CACHED ? 8 : 4) * (size_t)a.nK_pad;
     __shared__ int64_t red64[kSampleWarps];
-    __shared__ int32_t wcount[kSampleWarps];
+    __shared__ int32_t wtot[kSampleWarps];
 
     const int nK = a.nK;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto weight = [&](int b) -> int64_t { return CACHED ? Pw[b] : to_fixed48(ps[b]); };
 
     for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
         const float *prow = a.p + row * (int64_t)nK;
-        for (int b = tid; b < nK; b += kSampleThreads) {
-            ps[b] = prow[b];
-            sat[b] = 0;
+        // eight loads in flight per thread before any is used
+        for (int b0 = 0; b0 < nK; b0 += 8 * kSampleThreads) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int b = b0 + u * kSampleThreads + tid;
+                v[u] = b < nK ? __ldg(prow + b) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int b = b0 + u * kSampleThreads + tid;
+                if (b < nK) {
+                    if (CACHED) Pw[b] = to_fixed48(v[u]);
+                    else ps[b] = v[u];
+                    sat[b] = 0;
+                }
+            }
         }
         __syncthreads();
 
@@ -89,76 +121,92 @@ __global__ void __launch_bounds__(kSampleThreads)
 
         // ---- inclusion probabilities: exact water-filling ----------------
         int64_t R = a.M, T = 0;
-        const bool keep_all = a.M >= nK;
-        if (keep_all) {
+        if (a.M >= nK) {
             for (int b = tid; b < nK; b += kSampleThreads) sat[b] = 1;
             R = 0;
         } else {
+            // T = sum of the weights outside S; a round adds every b outside S
+            // with R * P_b >= T, i.e. P_b >= ceil(T / R) (positive integers),
+            // and carries T forward by subtracting what it added
+            int64_t local = 0;
+            for (int b = tid; b < nK; b += kSampleThreads) local += weight(b);
+            T = block_sum<int64_t>(local, red64);
             int64_t in_s = 0;
             for (int round = 0; round <= nK; ++round) {
                 R = a.M - in_s;
-                int64_t local = 0;
-                for (int b = tid; b < nK; b += kSampleThreads)
-                    if (!sat[b]) local += to_fixed48(ps[b]);
-                T = block_sum<int64_t>(local, red64);
                 if (T == 0 || R <= 0) break;
-                int64_t added = 0;
+                const int64_t thr = (T + R - 1) / R;
+                int64_t added = 0, added_w = 0;
                 for (int b = tid; b < nK; b += kSampleThreads) {
-                    if (!sat[b] && R * to_fixed48(ps[b]) >= T) {
+                    if (sat[b]) continue;
+                    const int64_t w = weight(b);
+                    if (w >= thr) {
                         sat[b] = 1;
                         ++added;
+                        added_w += w;
                     }
                 }
                 added = block_sum<int64_t>(added, red64);
                 if (added == 0) break;
+                added_w = block_sum<int64_t>(added_w, red64);
                 in_s += added;
+                T -= added_w;
             }
         }
         __syncthreads();
 
-        // ---- draws and ordered compaction -------------------------------
+        // ---- draws and ordered compaction: thread t owns blocks 4g..4g+3 --
         int32_t *idx_row = a.idx + row * (int64_t)a.capacity;
         float *logw_row = a.logw + row * (int64_t)a.capacity;
         int running = 0;
-        for (int base = 0; base < nK; base += kSampleThreads) {
-            const int b = base + tid;
-            bool take = false;
-            float lw = 0.0f;
-            if (b < nK) {
-                if (sat[b]) {
-                    take = true;
-                } else {
-                    const uint64_t RP = (uint64_t)(R * to_fixed48(ps[b]));
-                    if (RP != 0) {
-                        const uint4 u = philox4x32_10(
-                            make_uint4((uint32_t)(b >> 2), (uint32_t)i, (uint32_t)h, (uint32_t)beta),
-                            a.key0, a.key1);
-                        const int w = b & 3;
-                        const uint32_t U = w == 0 ? u.x : w == 1 ? u.y : w == 2 ? u.z : u.w;
-                        take = draw_below(U, (uint64_t)T, RP);
-                        if (take) {
-                            const double x = (double)(int64_t)RP / (double)T;
-                            lw = (float)(-log(x));
-                        }
+        for (int g0 = 0; 4 * g0 < nK; g0 += kSampleThreads) {
+            const int g = g0 + tid;
+            const int b0 = 4 * g;
+            bool take[4] = {false, false, false, false};
+            uint64_t rp[4] = {0, 0, 0, 0};
+            int cnt = 0;
+            if (b0 < nK) {
+                const uint4 u = philox4x32_10(
+                    make_uint4((uint32_t)g, (uint32_t)i, (uint32_t)h, (uint32_t)beta), a.key0, a.key1);
+                const uint32_t U[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int b = b0 + k;
+                    if (b >= nK) break;
+                    if (sat[b]) {
+                        take[k] = true;
+                    } else {
+                        rp[k] = (uint64_t)(R * weight(b));
+                        take[k] = rp[k] != 0 && draw_below(U[k], (uint64_t)T, rp[k]);
                     }
+                    cnt += take[k];
                 }
             }
-            const uint32_t ballot = __ballot_sync(0xffffffffu, take);
-            if (lane == 0) wcount[warp] = __popc(ballot);
+            // block-wide exclusive scan of the per-thread counts
+            int x = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) wtot[warp] = x;
             __syncthreads();
-            int before = 0, total = 0;
+            int pos = running + x - cnt, total = 0;
 #pragma unroll
             for (int w = 0; w < kSampleWarps; ++w) {
-                const int c = wcount[w];
-                before += w < warp ? c : 0;
+                const int c = wtot[w];
+                pos += w < warp ? c : 0;
                 total += c;
             }
-            if (take) {
-                const int pos = running + before + __popc(ballot & ((1u << lane) - 1u));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (!take[k]) continue;
                 if (pos < a.capacity) {
-                    idx_row[pos] = b;
-                    logw_row[pos] = lw;
+                    idx_row[pos] = b0 + k;
+                    logw_row[pos] =
+                        rp[k] ? (float)(-log((double)(int64_t)rp[k] / (double)T)) : 0.0f;
                 }
+                ++pos;
             }
             running += total;
             __syncthreads();
@@ -177,20 +225,28 @@ __global__ void __launch_bounds__(kSampleThreads)
 }  // namespace
 
 size_t sample_smem_bytes(int nK) {
-    const int nK_pad = (nK + 3) & ~3;
-    return sizeof(float) * (size_t)nK_pad + (size_t)nK_pad;
+    const size_t nK_pad = (size_t)((nK + 3) & ~3);
+    return (nK <= kCacheMaxBlocks ? 8 : 4) * nK_pad + nK_pad;
 }
 
 cudaError_t launch_sample(const SampleArgs &a, int num_sms, cudaStream_t stream) {
     const size_t smem = sample_smem_bytes(a.nK);
-    cudaError_t e = cudaFuncSetAttribute(sample_compact_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     int64_t grid = a.rows;
-    const int64_t cap = (int64_t)num_sms * 16;
+    const int64_t cap = (int64_t)num_sms * 64;
     if (grid > cap) grid = cap;
     if (grid < 1) return cudaSuccess;
-    sample_compact_kernel<<<(unsigned)grid, kSampleThreads, smem, stream>>>(a);
+    cudaError_t e;
+    if (a.nK <= kCacheMaxBlocks) {
+        e = cudaFuncSetAttribute(sample_compact_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        sample_compact_kernel<true><<<(unsigned)grid, kSampleThreads, smem, stream>>>(a);
+    } else {
+        e = cudaFuncSetAttribute(sample_compact_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        sample_compact_kernel<false><<<(unsigned)grid, kSampleThreads, smem, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -254,14 +254,41 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
             float acc[BPT];
 #pragma unroll
             for (int k = 0; k < BPT; ++k) acc[k] = 0.0f;
-            for (int j = 0; j < a.C; ++j) {
-                const float f = f_s[j];
-                if (f == 0.0f) continue;
-                const int64_t cj = row * a.C + j;
-                const float coef = f * ex2_approx(a.mref[cj * a.nT + T] - m_s[j]);
-                const float *rr = a.r + cj * a.ldr + (int64_t)T * BPT;
+            // four centroids at a time: all their loads in flight before use
+            for (int j0 = 0; j0 < a.C; j0 += 4) {
+                float mr[4], rv[4][BPT];
 #pragma unroll
-                for (int k = 0; k < BPT; ++k) acc[k] = fmaf(coef, rr[k], acc[k]);
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u;
+                    mr[u] = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < BPT; ++k) rv[u][k] = 0.0f;
+                    if (j < a.C) {
+                        const int64_t cj = row * a.C + j;
+                        mr[u] = __ldg(a.mref + cj * a.nT + T);
+                        const float *rr = a.r + cj * a.ldr + (int64_t)T * BPT;
+                        if constexpr (BPT % 4 == 0) {
+#pragma unroll
+                            for (int k = 0; k < BPT; k += 4) {
+                                const float4 q = __ldg(reinterpret_cast<const float4 *>(rr + k));
+                                rv[u][k] = q.x; rv[u][k + 1] = q.y; rv[u][k + 2] = q.z; rv[u][k + 3] = q.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < BPT; ++k) rv[u][k] = __ldg(rr + k);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = j0 + u;
+                    if (j >= a.C) break;
+                    const float f = f_s[j];
+                    if (f == 0.0f) continue;
+                    const float coef = f * ex2_approx(mr[u] - m_s[j]);
+#pragma unroll
+                    for (int k = 0; k < BPT; ++k) acc[k] = fmaf(coef, rv[u][k], acc[k]);
+                }
             }
 #pragma unroll
             for (int k = 0; k < BPT; ++k) {
