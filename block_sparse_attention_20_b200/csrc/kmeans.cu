@@ -12,7 +12,8 @@
 //     32w..32w+31; the argmin (ties to the lower index) is reduced across the
 //     four lanes that share a row;
 //   - update: a stable counting sort of the rows by cluster (warp ballots),
-//     then thread x sums dimension x of each cluster's rows in ascending row
+//     then thread x sums dimension x of each cluster's rows as four
+//     interleaved partial sums in ascending row order, combined in a fixed
 //     order (deterministic), centroid = sum / size.
 //
 // Rules (open in the abstract, fixed here): C_eff = min(C, n) clusters;
@@ -97,10 +98,14 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                 chi[j * LDQ + x] = h;
                 clo[j * LDQ + x] = __float2bfloat16_rn(c - __bfloat162float(h));
             }
-            if (tid < kMaxC) {
+            // squared norms: warp w takes centroids w, w+4, ...; lanes split the dimensions
+            for (int j = warp; j < kMaxC; j += 4) {
                 float s = 0.0f;
-                for (int x = 0; x < D; ++x) s = fmaf(cent[tid * D + x], cent[tid * D + x], s);
-                cnorm[tid] = s;
+#pragma unroll
+                for (int x = lane; x < D; x += 32) s = fmaf(cent[j * D + x], cent[j * D + x], s);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0) cnorm[j] = s;
             }
             __syncthreads();
 
@@ -188,10 +193,21 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                 for (int j = 0; j < ce; ++j) {
                     const int c = cnt_s[j];
                     if (c == 0) continue;
-                    float s = 0.0f;
+                    // four interleaved partial sums (rows e = 0,4,8,.. / 1,5,9,.. / ...)
+                    // in ascending row order each, combined in a fixed order
+                    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
                     const int b0 = base_s[j];
-                    for (int e = 0; e < c; ++e) s += __bfloat162float(qs[order_s[b0 + e] * LDQ + x]);
-                    cent[j * D + x] = s / (float)c;
+                    int e = 0;
+                    for (; e + 4 <= c; e += 4) {
+                        s0 += __bfloat162float(qs[order_s[b0 + e] * LDQ + x]);
+                        s1 += __bfloat162float(qs[order_s[b0 + e + 1] * LDQ + x]);
+                        s2 += __bfloat162float(qs[order_s[b0 + e + 2] * LDQ + x]);
+                        s3 += __bfloat162float(qs[order_s[b0 + e + 3] * LDQ + x]);
+                    }
+                    if (e < c) s0 += __bfloat162float(qs[order_s[b0 + e] * LDQ + x]);
+                    if (e + 1 < c) s1 += __bfloat162float(qs[order_s[b0 + e + 1] * LDQ + x]);
+                    if (e + 2 < c) s2 += __bfloat162float(qs[order_s[b0 + e + 2] * LDQ + x]);
+                    cent[j * D + x] = ((s0 + s1) + (s2 + s3)) / (float)c;
                 }
             }
             __syncthreads();
