@@ -312,6 +312,7 @@ def main():
         "clocks": clk.summary(),
     }
 
+    line["keep_all"] = keep_all(abatt, cfg, Q, K, V, w, O, ws_att, stream)
     if not args.no_e2e:
         line["e2e"] = e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world)
     if rank == 0 and not args.no_cpu_baseline:
@@ -321,6 +322,33 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def keep_all(abatt, cfg, Q, K, V, w, O, ws, stream):
+    """The same attention kernel fed every key block with weight 1 (dense
+    attention through the gather path), timed the same way."""
+    import torch
+
+    rows, nK = w.rows, w.nK
+    counts = torch.full((rows,), nK, dtype=torch.int32, device=Q.device)
+    idx = torch.arange(nK, dtype=torch.int32, device=Q.device).repeat(rows, 1)
+    logw = torch.zeros((rows, nK), dtype=torch.float32, device=Q.device)
+    for _ in range(2):
+        abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    reps = 3
+    a.record(stream)
+    for _ in range(reps):
+        abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    dense = 4.0 * w.B * w.H * w.N * w.N * w.d
+    tiles = rows * ((nK + 128 // w.Bk - 1) // (128 // w.Bk))
+    return {"attention_ms": ms, "dense_tflops": dense / (ms * 1e-3) / 1e12,
+            "executed_tflops": tiles * 4.0 * 128 * 128 * w.d / (ms * 1e-3) / 1e12}
 
 
 def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):

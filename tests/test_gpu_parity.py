@@ -327,6 +327,15 @@ def test_forward_wan1_3b_sampled_rows():
     _forward_check(w, rows, heads=heads)
 
 
+def test_forward_hunyuan_sampled_rows():
+    # 118,800 tokens: 929 query blocks per head (odd, last block 16 rows)
+    w = synth.HUNYUAN
+    heads = 4
+    nQ = w.nQ
+    rows = [h * nQ + i for h, i in [(0, 0), (0, nQ - 1), (1, 464), (2, 928), (3, 3)]]
+    _forward_check(w, rows, heads=heads)
+
+
 def test_forward_wan14b_full_size_sampled_rows():
     w = synth.WAN_14B
     nQ = w.nQ
