@@ -24,16 +24,17 @@
 //   warp 1      tensor-memory owner and tcgen05 MMA issuer:
 //               S_s = Q_s K^T (fp32, 128 TMEM columns per row),
 //               O_s += P_s V  (P_s read back from the columns S_s used);
-//   warps 2-17  softmax, four warpgroups: row s of the pair and column half
-//               hh of each tile per warpgroup (thread = query): raw per-block
-//               maxima of its 64 columns, the two halves' tile maxima of
-//               s*log2(e)*S + log-weight (base 2) exchanged through shared
-//               memory, lazy running maximum (O is rescaled only when it grows
-//               by more than 8), P in bf16 back into tensor memory, final
-//               O / l to bf16 (each half writes its 64 output columns).
+//   warps 2-17  softmax, eight warps per row s of the pair; a warp owns 16
+//               query rows of its tensor-memory lane quarter and its two
+//               half-warps split each row's 128 columns (two threads per
+//               query): raw per-block maxima of the thread's 64 columns, the
+//               row's tile maximum of s*log2(e)*S + log-weight (base 2) by one
+//               shuffle, lazy running maximum (O is rescaled only when it
+//               grows by more than 8), P in bf16 back into tensor memory,
+//               final O / l to bf16 (each thread writes half of its row).
 //               The softmax latency of a tile sits on each row's critical
 //               path (P replaces S in tensor memory, so S(t+1) waits for
-//               PV(t)); splitting the columns halves it.
+//               PV(t)); two threads per row halve it.
 #include "kernels.cuh"
 
 namespace abatt {
@@ -177,9 +178,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __shared__ __align__(8) uint64_t bar_drain;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
-    __shared__ float xchg[2][2][2][128];  // [row s][tile parity][column half][query]
-    __shared__ float xsum[2][2][128];      // [row s][column half][query] row sums
-    __shared__ __align__(8) uint64_t bar_x[2];  // the two halves of row s have exchanged
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT))
@@ -201,8 +199,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&bar_kve[s], 1);
         }
         mbar_init(&bar_drain, 1);
-        mbar_init(&bar_x[0], 8);
-        mbar_init(&bar_x[1], 8);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -366,24 +362,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp >= 2) {
         // ================================ softmax =====================================
+        // Eight warps per row of the pair.  A warp owns 16 query rows (TMEM
+        // lanes) of its lane quarter; the two half-warps split each row's
+        // columns, so a row's maximum and sum need one shuffle, not a barrier.
         constexpr int HB = BPT >= 2 ? BPT / 2 : 1;  // blocks (or block parts) per column half
         const int sw = warp - 2;
-        const int s = sw >> 3;         // row of the pair
-        const int hh = (sw >> 2) & 1;  // column half of each tile
-        const int wq = warp & 3;       // tensor-memory lane quarter
-        const int r = wq * 32 + lane;  // query row within the block == TMEM lane
-        const uint32_t t_lane = (uint32_t)(wq * 32) << 16;
+        const int s = sw >> 3;              // row of the pair
+        const int sub = (sw >> 2) & 1;      // 16-lane half of the lane quarter
+        const int wq = warp & 3;            // tensor-memory lane quarter
+        const int hh = lane >> 4;           // column half of each tile
+        const int r = wq * 32 + sub * 16 + (lane & 15);  // query row within the block == TMEM lane
+        const uint32_t t_lane = (uint32_t)(wq * 32 + sub * 16) << 16;
         const uint32_t s_col = tmem + t_lane + s * 128;
         const uint32_t o_col = tmem + t_lane + 256 + s * 128;
-        uint32_t s_uses = 0, o_uses = 0, x_uses = 0;
-        // both halves of the row have published their values (bounded wait)
-        auto exchange = [&]() -> bool {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_x[s]);
-            const bool got = mbar_wait(&bar_x[s], x_uses & 1, wc, 0x20b);
-            ++x_uses;
-            return got;
-        };
+        uint32_t s_uses = 0, o_uses = 0;
         bool ok = true;
         for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
             int64_t rr[2];
@@ -424,7 +416,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tc_fence_after();
                 uint32_t v[2][32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) tmem_ld32(s_col + hh * 64 + c * 32, v[c]);
+                for (int c = 0; c < 2; ++c) tmem_ld32_split<64>(s_col + c * 32, v[c]);
                 tmem_wait_ld();
                 // column (within the tile) of v[c][j]: 64*hh + 32*c + j; its block
                 // slot within this half: (32c + j) / BK (or 0 for blocks wider
@@ -445,20 +437,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
+                    for (int j = 0; j < 32; j += 2) {
                         const int k = BPT >= 2 ? (c * 32 + j) / BK : 0;
-                        bmax[k] = fmaxf(bmax[k], __uint_as_float(v[c][j]));
+                        bmax[k] = fmax3f(bmax[k], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
                     }
                 float hmax = kNegInf;
 #pragma unroll
                 for (int k = 0; k < HB; ++k) hmax = fmaxf(hmax, fmaf(bmax[k], a.scale_log2, bias[k]));
-                // both halves' S reads are done once the exchange completes, so P
-                // may then overwrite S anywhere in the row's columns
-                xchg[s][t & 1][hh][r] = hmax;
-                tc_fence_before();
-                if (!exchange()) { ok = false; break; }
-                tc_fence_after();
-                const float tmax = fmaxf(hmax, xchg[s][t & 1][hh ^ 1][r]);
+                const float tmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, 16));
                 const bool need = tmax > m_run + kRescaleThreshold;
                 const float m_use = need ? tmax : m_run;
                 const float alpha = need ? ((m_run == kNegInf) ? 0.0f : ex2_approx(m_run - tmax)) : 1.0f;
@@ -478,20 +464,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         rs += p0 + p1;
                         pk[j >> 1] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(s_col + hh * 32 + c * 16, pk);
+                    // P (bf16 pairs) over the row's S: this half's keys 64*hh + 32c + 0..31
+                    // go to packed columns 32*hh + 16c + 0..15; both halves of the warp
+                    // finished reading S above
+                    tmem_st16_split<32>(s_col + c * 16, pk);
                 }
-                // rescale this half's O columns (after P, so the scores are
-                // dead): the commit that signalled S(t) covers the previous PV
+                // rescale this row's O (after P, so the scores are dead): the
+                // commit that signalled S(t) covers the previous PV
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
                     for (int c = 0; c < D / 64; ++c) {
                         uint32_t o[32];
-                        const uint32_t oa = o_col + hh * (D / 2) + c * 32;
-                        tmem_ld32(oa, o);
+                        const uint32_t oa = o_col + c * 32;
+                        tmem_ld32_split<D / 2>(oa, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st32(oa, o);
+                        tmem_st32_split<D / 2>(oa, o);
                     }
                 }
                 tmem_wait_st();
@@ -511,10 +500,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 continue;
             }
-            // epilogue: the row sum is split over the two halves
-            xsum[s][hh][r] = l;
-            if (!exchange()) { ok = false; break; }
-            l += xsum[s][hh ^ 1][r];
+            // epilogue: the row sum is split over the two half-warps
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
             if (!mbar_wait(&bar_of[s], o_uses & 1, wc, 0x209)) { ok = false; break; }
             ++o_uses;
             tc_fence_after();
@@ -522,7 +509,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
                 uint32_t o[32];
-                tmem_ld32(o_col + hh * (D / 2) + c * 32, o);
+                tmem_ld32_split<D / 2>(o_col + c * 32, o);
                 tmem_wait_ld();
                 if (r < nrows) {
 #pragma unroll
