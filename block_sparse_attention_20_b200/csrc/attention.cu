@@ -288,77 +288,80 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp == 1) {
         // ================================ MMA issuer ==================================
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16(128, 128);
-            constexpr uint32_t idesc_o = idesc_bf16(128, D, /*b_mn_major=*/true);
-            uint32_t rp = 0;  // ring position of K(t); V(t) is rp+1
-            uint32_t q_uses[2] = {0, 0}, pv_ops[2] = {0, 0}, o_items[2] = {0, 0};
-            bool ok = true;
-            const uint32_t q_addr0 = smem_u32(sQ), ring_addr = smem_u32(sRing);  // < 256 KB: the
-            // 14-bit address field of a descriptor never carries into the next field
-            auto op_s = [&](int s, uint32_t kpos, bool release, bool last) -> bool {
-                const int stg = kpos % ST;
-                if (!mbar_wait(&bar_kvf[stg], (kpos / ST) & 1, wc, 0x203)) return false;
-                tc_fence_after();
-                // descriptors built once per op; each k-step adds its byte offset / 16
-                const uint64_t qd = sdesc_sw128(q_addr0 + s * TILE, 16, 1024);
-                const uint64_t kd = sdesc_sw128(ring_addr + stg * TILE, 16, KFOLD ? CH * 1024 : 1024);
+        // The whole warp runs the schedule, so its control flow and the
+        // descriptors stay warp-uniform; one elected lane issues each tcgen05
+        // instruction.
+        constexpr uint32_t idesc_s = idesc_bf16(128, 128);
+        constexpr uint32_t idesc_o = idesc_bf16(128, D, /*b_mn_major=*/true);
+        uint32_t rp = 0;  // ring position of K(t); V(t) is rp+1
+        uint32_t q_uses[2] = {0, 0}, pv_ops[2] = {0, 0}, o_items[2] = {0, 0};
+        bool ok = true;
+        const uint32_t q_addr0 = smem_u32(sQ), ring_addr = smem_u32(sRing);  // < 256 KB: the
+        // 14-bit address field of a descriptor never carries into the next field
+        auto wait_all = [&](uint64_t *bar, uint32_t parity, uint32_t site) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc, site));
+        };
+        auto op_s = [&](int s, uint32_t kpos, bool release, bool last) -> bool {
+            const int stg = kpos % ST;
+            if (!wait_all(&bar_kvf[stg], (kpos / ST) & 1, 0x203)) return false;
+            tc_fence_after();
+            // descriptors built once per op; each k-step adds its byte offset / 16
+            const uint64_t qd = sdesc_sw128(q_addr0 + s * TILE, 16, 1024);
+            const uint64_t kd = sdesc_sw128(ring_addr + stg * TILE, 16, KFOLD ? CH * 1024 : 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    const uint32_t koff =
-                        KFOLD ? (kk >> 2) * 1024 + (kk & 3) * 32 : (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_bf16_ss(tmem + s * 128, qd + (qoff >> 4), kd + (koff >> 4), idesc_s, kk > 0);
-                }
-                if (release) umma_commit(&bar_kve[stg]);
-                umma_commit(&bar_sf[s]);
-                if (last) umma_commit(&bar_qe[s]);
-                return true;
-            };
-            auto op_pv = [&](int s, uint32_t vpos, int t, bool release, bool last) -> bool {
-                if (!mbar_wait(&bar_pf[s], pv_ops[s] & 1, wc, 0x204)) return false;
-                if (t == 0 && o_items[s] > 0 &&
-                    !mbar_wait(&bar_oe[s], (o_items[s] - 1) & 1, wc, 0x205))
-                    return false;
-                const int stg = vpos % ST;
-                if (!mbar_wait(&bar_kvf[stg], (vpos / ST) & 1, wc, 0x206)) return false;
-                tc_fence_after();
-                const uint64_t vd = sdesc_sw128(ring_addr + stg * TILE, BK * 128, 1024);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t boff = (uint32_t)((16 * j) / BK) * BLK + (uint32_t)((16 * j) % BK) * 128;
-                    umma_bf16_ts(tmem + 256 + s * 128, tmem + s * 128 + j * 8, vd + (boff >> 4), idesc_o,
-                                 (t > 0 || j > 0) ? 1u : 0u);
-                }
-                if (release) umma_commit(&bar_kve[stg]);
-                if (last) {
-                    umma_commit(&bar_of[s]);
-                    ++o_items[s];
-                }
-                ++pv_ops[s];
-                return true;
-            };
-            for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
-                const int U = a.ulen[pr];
-                const int n = (U + BPT - 1) / BPT;
-                if (n == 0) continue;
-                int64_t rr[2];
-                pair_rows(pr, a.nQ, &rr[0], &rr[1]);
-                const bool has1 = rr[1] >= 0;
-                for (int s = 0; ok && s < (has1 ? 2 : 1); ++s) {
-                    if (!mbar_wait(&bar_qf[s], q_uses[s] & 1, wc, 0x207)) ok = false;
-                    ++q_uses[s];
-                }
-                const uint32_t base = rp;
-                for (int t = 0; ok && t <= n; ++t) {
-                    const uint32_t kp = base + 2 * t, vp_prev = base + 2 * (t - 1) + 1, vp = kp + 1;
-                    if (t < n && !op_s(0, kp, !has1, t == n - 1)) ok = false;
-                    if (ok && has1 && t >= 1 && !op_pv(1, vp_prev, t - 1, true, t - 1 == n - 1)) ok = false;
-                    if (ok && has1 && t < n && !op_s(1, kp, true, t == n - 1)) ok = false;
-                    if (ok && t < n && !op_pv(0, vp, t, !has1, t == n - 1)) ok = false;
-                }
-                rp = base + 2 * n;
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                const uint32_t koff =
+                    KFOLD ? (kk >> 2) * 1024 + (kk & 3) * 32 : (kk >> 2) * 16384 + (kk & 3) * 32;
+                umma_bf16_ss_w(tmem + s * 128, qd + (qoff >> 4), kd + (koff >> 4), idesc_s, kk > 0);
             }
+            if (release) umma_commit_w(&bar_kve[stg]);
+            umma_commit_w(&bar_sf[s]);
+            if (last) umma_commit_w(&bar_qe[s]);
+            return true;
+        };
+        auto op_pv = [&](int s, uint32_t vpos, int t, bool release, bool last) -> bool {
+            if (!wait_all(&bar_pf[s], pv_ops[s] & 1, 0x204)) return false;
+            if (t == 0 && o_items[s] > 0 && !wait_all(&bar_oe[s], (o_items[s] - 1) & 1, 0x205))
+                return false;
+            const int stg = vpos % ST;
+            if (!wait_all(&bar_kvf[stg], (vpos / ST) & 1, 0x206)) return false;
+            tc_fence_after();
+            const uint64_t vd = sdesc_sw128(ring_addr + stg * TILE, BK * 128, 1024);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t boff = (uint32_t)((16 * j) / BK) * BLK + (uint32_t)((16 * j) % BK) * 128;
+                umma_bf16_ts_w(tmem + 256 + s * 128, tmem + s * 128 + j * 8, vd + (boff >> 4), idesc_o,
+                               (t > 0 || j > 0) ? 1u : 0u);
+            }
+            if (release) umma_commit_w(&bar_kve[stg]);
+            if (last) {
+                umma_commit_w(&bar_of[s]);
+                ++o_items[s];
+            }
+            ++pv_ops[s];
+            return true;
+        };
+        for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
+            const int U = __shfl_sync(0xffffffffu, a.ulen[pr], 0);
+            const int n = (U + BPT - 1) / BPT;
+            if (n == 0) continue;
+            int64_t rr[2];
+            pair_rows(pr, a.nQ, &rr[0], &rr[1]);
+            const bool has1 = rr[1] >= 0;
+            for (int s = 0; ok && s < (has1 ? 2 : 1); ++s) {
+                if (!wait_all(&bar_qf[s], q_uses[s] & 1, 0x207)) ok = false;
+                ++q_uses[s];
+            }
+            const uint32_t base = rp;
+            for (int t = 0; ok && t <= n; ++t) {
+                const uint32_t kp = base + 2 * t, vp_prev = base + 2 * (t - 1) + 1, vp = kp + 1;
+                if (t < n && !op_s(0, kp, !has1, t == n - 1)) ok = false;
+                if (ok && has1 && t >= 1 && !op_pv(1, vp_prev, t - 1, true, t - 1 == n - 1)) ok = false;
+                if (ok && has1 && t < n && !op_s(1, kp, true, t == n - 1)) ok = false;
+                if (ok && t < n && !op_pv(0, vp, t, !has1, t == n - 1)) ok = false;
+            }
+            rp = base + 2 * n;
         }
     } else if (warp >= 2) {
         // ================================ softmax =====================================
