@@ -301,9 +301,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         auto wait_all = [&](uint64_t *bar, uint32_t parity, uint32_t site) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc, site));
         };
-        auto op_s = [&](int s, uint32_t kpos, bool release, bool last) -> bool {
+        // K(t) / V(t) have landed (called before the waits that gate issue)
+        auto wait_kv = [&](uint32_t pos, uint32_t site) -> bool {
+            return wait_all(&bar_kvf[pos % ST], (pos / ST) & 1, site);
+        };
+        auto op_s = [&](int s, uint32_t kpos, bool release, bool last) {
             const int stg = kpos % ST;
-            if (!wait_all(&bar_kvf[stg], (kpos / ST) & 1, 0x203)) return false;
             tc_fence_after();
             // descriptors built once per op; each k-step adds its byte offset / 16
             const uint64_t qd = sdesc_sw128(q_addr0 + s * TILE, 16, 1024);
@@ -318,14 +321,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (release) umma_commit_w(&bar_kve[stg]);
             umma_commit_w(&bar_sf[s]);
             if (last) umma_commit_w(&bar_qe[s]);
-            return true;
         };
         auto op_pv = [&](int s, uint32_t vpos, int t, bool release, bool last) -> bool {
-            if (!wait_all(&bar_pf[s], pv_ops[s] & 1, 0x204)) return false;
             if (t == 0 && o_items[s] > 0 && !wait_all(&bar_oe[s], (o_items[s] - 1) & 1, 0x205))
                 return false;
+            if (!wait_all(&bar_pf[s], pv_ops[s] & 1, 0x204)) return false;
             const int stg = vpos % ST;
-            if (!wait_all(&bar_kvf[stg], (vpos / ST) & 1, 0x206)) return false;
             tc_fence_after();
             const uint64_t vd = sdesc_sw128(ring_addr + stg * TILE, BK * 128, 1024);
 #pragma unroll
@@ -354,12 +355,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 ++q_uses[s];
             }
             const uint32_t base = rp;
-            for (int t = 0; ok && t <= n; ++t) {
-                const uint32_t kp = base + 2 * t, vp_prev = base + 2 * (t - 1) + 1, vp = kp + 1;
-                if (t < n && !op_s(0, kp, !has1, t == n - 1)) ok = false;
-                if (ok && has1 && t >= 1 && !op_pv(1, vp_prev, t - 1, true, t - 1 == n - 1)) ok = false;
-                if (ok && has1 && t < n && !op_s(1, kp, true, t == n - 1)) ok = false;
-                if (ok && t < n && !op_pv(0, vp, t, !has1, t == n - 1)) ok = false;
+            // issue order: S0(0) S1(0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ...
+            // Each row's chain is softmax(t) -> PV(t) -> S(t+1) (S(t+1) overwrites
+            // the P(t) that PV(t) reads; tcgen05 MMAs of one thread run in issue
+            // order).  Waits for K/V data sit before the wait on P, so once P is
+            // ready nothing else delays the two MMAs of its row.
+            if (!wait_kv(base, 0x203)) ok = false;
+            if (ok) op_s(0, base, !has1, n == 1);
+            if (ok && has1) op_s(1, base, true, n == 1);
+            for (int t = 0; ok && t < n; ++t) {
+                const uint32_t kp = base + 2 * t, vp = kp + 1, kn = kp + 2;
+                const bool more = t + 1 < n;
+                if (!wait_kv(vp, 0x206) || (more && !wait_kv(kn, 0x203))) { ok = false; break; }
+                if (!op_pv(0, vp, t, !has1, !more)) { ok = false; break; }
+                if (more) op_s(0, kn, !has1, t + 1 == n - 1);
+                if (has1) {
+                    if (!op_pv(1, vp, t, true, !more)) { ok = false; break; }
+                    if (more) op_s(1, kn, true, t + 1 == n - 1);
+                }
             }
             rp = base + 2 * n;
         }

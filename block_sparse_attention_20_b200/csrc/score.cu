@@ -117,27 +117,32 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else if (warp == 9) {
         // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0 && mbar_wait(&bar_a, 0, wc, 0x102)) {
+        // the whole warp follows the schedule (warp-uniform control flow and
+        // descriptors); one elected lane issues each tcgen05 instruction
+        auto wait_all = [&](uint64_t *bar, uint32_t parity, uint32_t site) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc, site));
+        };
+        if (wait_all(&bar_a, 0, 0x102)) {
             tc_fence_after();
             constexpr uint32_t idesc = idesc_bf16(128, 128);
             const uint32_t a_hi = smem_u32(sA_hi), a_lo = smem_u32(sA_lo);
+            const uint64_t dhi = sdesc_sw128(a_hi, 16, 1024), dlo = sdesc_sw128(a_lo, 16, 1024);
+            const bool use_lo = a.use_lo != 0;
             for (int kt = 0; kt < a.nT; ++kt) {
                 const int s = kt % ST, buf = kt & 1, use = kt >> 1;
-                if (!mbar_wait(&bar_kfull[s], (kt / ST) & 1, wc, 0x103)) break;
-                if (use > 0 && !mbar_wait(&bar_sempty[buf], (use - 1) & 1, wc, 0x104)) break;
+                if (!wait_all(&bar_kfull[s], (kt / ST) & 1, 0x103)) break;
+                if (use > 0 && !wait_all(&bar_sempty[buf], (use - 1) & 1, 0x104)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * 128;
-                const uint32_t kb = smem_u32(sK + s * TILE);
+                const uint64_t kd = sdesc_sw128(smem_u32(sK + s * TILE), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    const uint64_t bdesc = sdesc_sw128(kb + off, 16, 1024);
-                    umma_bf16_ss(d_tmem, sdesc_sw128(a_hi + off, 16, 1024), bdesc, idesc, kk > 0);
-                    if (a.use_lo)
-                        umma_bf16_ss(d_tmem, sdesc_sw128(a_lo + off, 16, 1024), bdesc, idesc, 1);
+                    const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                    umma_bf16_ss_w(d_tmem, dhi + off, kd + off, idesc, kk > 0);
+                    if (use_lo) umma_bf16_ss_w(d_tmem, dlo + off, kd + off, idesc, 1);
                 }
-                umma_commit(&bar_kempty[s]);
-                umma_commit(&bar_sfull[buf]);
+                umma_commit_w(&bar_kempty[s]);
+                umma_commit_w(&bar_sfull[buf]);
                 committed = kt;
             }
         }
