@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--budget-bp", type=int, default=None, help="override (10000 = keep-all)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-keep-all", action="store_true", help="skip the keep-all attention timing")
     return ap.parse_args()
 
 
@@ -312,7 +313,8 @@ def main():
         "clocks": clk.summary(),
     }
 
-    line["keep_all"] = keep_all(abatt, cfg, Q, K, V, w, O, ws_att, stream)
+    if not args.no_keep_all:
+        line["keep_all"] = keep_all(abatt, cfg, Q, K, V, w, O, ws_att, stream)
     if not args.no_e2e:
         line["e2e"] = e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world)
     if rank == 0 and not args.no_cpu_baseline:

@@ -22,6 +22,30 @@ struct Geom {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The scoring kernel runs one CTA per (centroid tile, head, key-range chunk),
+// one CTA per SM at a time.  Split the key tiles into the fewest chunks (at
+// most kMaxScoreChunks, each of at least 24 tiles) whose CTA count fills its
+// last wave of SMs to 95 %, else take the best fill found.
+constexpr int kMaxScoreChunks = 8;
+void score_chunks(int nT, int64_t ctas, int sms, int *nchunk, int *chunk_tiles) {
+    const int nmax = nT / 24 < 1 ? 1 : (nT / 24 > kMaxScoreChunks ? kMaxScoreChunks : nT / 24);
+    int best = 1;
+    double best_fill = 0.0;
+    for (int n = 1; n <= nmax; ++n) {
+        const int per = (nT + n - 1) / n;
+        const int neff = (nT + per - 1) / per;  // no empty chunk
+        const double waves = (double)(ctas * neff) / (sms > 0 ? sms : 1);
+        const double fill = waves / ceil(waves);
+        if (fill > best_fill + 1e-9) {
+            best_fill = fill;
+            best = n;
+        }
+        if (fill >= 0.95) break;
+    }
+    *chunk_tiles = (nT + best - 1) / best;
+    *nchunk = (nT + *chunk_tiles - 1) / *chunk_tiles;
+}
+
 abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (!s || !c) return ABATT_ERR_INVALID_ARG;
     if (s->B <= 0 || s->H <= 0 || s->N <= 0 || s->d <= 0) return ABATT_ERR_INVALID_ARG;
@@ -70,7 +94,7 @@ Layout layout(abatt_call call, const Geom &g) {
         L.weight = off;  off = align256(off + crow * 4);
         L.r = off;       off = align256(off + crow * g.ldr * 4);
         L.mref = off;    off = align256(off + crow * g.nT * 4);
-        L.mz = off;      off = align256(off + crow * 8);
+        L.mz = off;      off = align256(off + crow * 8 * kMaxScoreChunks);
     }
     if (call == ABATT_CALL_ATTENTION || call == ABATT_CALL_FORWARD) {
         const size_t pairs = (size_t)pairs_of(g);
@@ -192,6 +216,7 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     ScoreArgs sa;
     sa.heads = (int)g.heads; sa.N = g.N; sa.D = g.d; sa.Bk = g.Bk; sa.MC = (int)MC;
     sa.nT = g.nT; sa.ldr = g.ldr; sa.use_lo = 1;
+    score_chunks(g.nT, ((int)MC + 127) / 128 * g.heads, sms, &sa.nchunk, &sa.chunk_tiles);
     sa.r = at<float>(ws, L.r);
     sa.mref = at<float>(ws, L.mref);
     sa.mz = at<float2>(ws, L.mz);
@@ -203,6 +228,7 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     CombineArgs ca;
     ca.rows = g.rows; ca.C = g.C; ca.nK = g.nK; ca.nT = g.nT; ca.ldr = g.ldr; ca.Bk = g.Bk;
     ca.r = sa.r; ca.mref = sa.mref; ca.weight = ka.weight; ca.mz = sa.mz; ca.p = p;
+    ca.nchunk = sa.nchunk;
     return cuda_status(launch_combine(ca, sms, st));
 }
 

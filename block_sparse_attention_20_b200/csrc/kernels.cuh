@@ -32,9 +32,11 @@ struct ScoreArgs {
     int nT;        // key tiles per head, ceil(N/128)
     int ldr;       // row stride of r in floats (nT * 128/Bk)
     int use_lo;    // add the lo half of the split centroids (fp32-accurate logits)
+    int nchunk;    // the key tiles are split into nchunk ranges of chunk_tiles (one CTA each)
+    int chunk_tiles;
     float *r;      // [heads*MC][ldr]
-    float *mref;   // [heads*MC][nT]
-    float2 *mz;    // [heads*MC] (final max, sum) in base 2
+    float *mref;   // [heads*MC][nT], running maximum within the tile's chunk
+    float2 *mz;    // [heads*MC][nchunk] (max, sum) of each chunk in base 2
     WsHeader *hdr;
     uint64_t wait_ns;
 };
@@ -47,7 +49,7 @@ cudaError_t launch_score(const ScoreArgs &a, const ScoreMaps &maps, int num_sms,
 // Combine the C centroids of each query block into p (see score.cu).
 struct CombineArgs {
     int64_t rows;  // query blocks
-    int C, nK, nT, ldr, Bk;
+    int C, nK, nT, ldr, Bk, nchunk;
     const float *r, *mref, *weight;
     const float2 *mz;
     float *p;      // [rows][nK]

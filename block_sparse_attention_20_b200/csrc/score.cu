@@ -65,7 +65,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     __shared__ float2 mz_s[128];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mt = blockIdx.x, hd = blockIdx.y;
+    const int mt = blockIdx.x, hd = blockIdx.y, chunk = blockIdx.z;
+    // this CTA's key tiles: [kt0, kt0 + ntl)
+    const int kt0 = chunk * a.chunk_tiles;
+    const int ntl = min(a.chunk_tiles, a.nT - kt0);
     // a bounded wait elsewhere already gave up: do not start more work
     if (a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT))
         return;
@@ -106,13 +109,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 tma_load_3d(sA_hi + c * 16384, &maps.a_hi, &bar_a, c * 64, mt * 128, hd);
                 if (a.use_lo) tma_load_3d(sA_lo + c * 16384, &maps.a_lo, &bar_a, c * 64, mt * 128, hd);
             }
-            for (int kt = 0; kt < a.nT; ++kt) {
-                const int s = kt % ST;
-                if (kt >= ST && !mbar_wait(&bar_kempty[s], ((kt / ST) - 1) & 1, wc, 0x101)) break;
+            for (int i = 0; i < ntl; ++i) {
+                const int s = i % ST;
+                if (i >= ST && !mbar_wait(&bar_kempty[s], ((i / ST) - 1) & 1, wc, 0x101)) break;
                 mbar_arrive_expect_tx(&bar_kfull[s], TILE);
                 for (int c = 0; c < CH; ++c)
-                    tma_load_3d(sK + s * TILE + c * 16384, &maps.k, &bar_kfull[s], c * 64, kt * 128, hd);
-                issued = kt + 1;
+                    tma_load_3d(sK + s * TILE + c * 16384, &maps.k, &bar_kfull[s], c * 64, (kt0 + i) * 128, hd);
+                issued = i + 1;
             }
         }
     } else if (warp == 9) {
@@ -128,9 +131,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             const uint32_t a_hi = smem_u32(sA_hi), a_lo = smem_u32(sA_lo);
             const uint64_t dhi = sdesc_sw128(a_hi, 16, 1024), dlo = sdesc_sw128(a_lo, 16, 1024);
             const bool use_lo = a.use_lo != 0;
-            for (int kt = 0; kt < a.nT; ++kt) {
-                const int s = kt % ST, buf = kt & 1, use = kt >> 1;
-                if (!wait_all(&bar_kfull[s], (kt / ST) & 1, 0x103)) break;
+            for (int i = 0; i < ntl; ++i) {
+                const int s = i % ST, buf = i & 1, use = i >> 1;
+                if (!wait_all(&bar_kfull[s], (i / ST) & 1, 0x103)) break;
                 if (use > 0 && !wait_all(&bar_sempty[buf], (use - 1) & 1, 0x104)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + buf * 128;
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 }
                 umma_commit_w(&bar_kempty[s]);
                 umma_commit_w(&bar_sfull[buf]);
-                committed = kt;
+                committed = i;
             }
         }
     } else {
@@ -155,8 +158,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const bool valid = grow < a.MC;
         const int64_t gr = (int64_t)hd * a.MC + grow;
         float m_run = kNegInf, Z = 0.0f;
-        for (int kt = e; kt < a.nT; kt += 2) {
-            const int use = kt >> 1;
+        for (int i = e; i < ntl; i += 2) {
+            const int kt = kt0 + i, use = i >> 1;
             if (!mbar_wait(&bar_sfull[e], use & 1, wc, 0x105)) break;
             tc_fence_after();
             uint32_t v[4][32];
@@ -172,16 +175,19 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
             const int kbase = kt * 128;
             const int nvalid = min(128, a.N - kbase);
+            if (nvalid < 128) {  // the sequence's last tile: keys past N count for nothing
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (q * 32 + c >= nvalid) v[q][c] = __float_as_uint(kNegInf);
+            }
             float tm = kNegInf;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    float x = __uint_as_float(v[q][c]);
-                    if (q * 32 + c >= nvalid) x = kNegInf;
-                    v[q][c] = __float_as_uint(x);
-                    tm = fmaxf(tm, x);
-                }
+                for (int c = 0; c < 32; c += 2)
+                    tm = fmax3f(tm, __uint_as_float(v[q][c]), __uint_as_float(v[q][c + 1]));
             const float m_new = fmaxf(m_run, tm);
             const float alpha = (m_run == kNegInf) ? 0.0f : ex2_approx(m_run - m_new);
             Z *= alpha;
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             const float m = fmaxf(m_run, o.x);
             const float z0 = (m_run == kNegInf) ? 0.0f : Z * ex2_approx(m_run - m);
             const float z1 = (o.x == kNegInf) ? 0.0f : o.y * ex2_approx(o.x - m);
-            if (valid) a.mz[gr] = make_float2(m, z0 + z1);
+            if (valid) a.mz[gr * a.nchunk + chunk] = make_float2(m, z0 + z1);
         }
     }
     if (warp >= 8) {
@@ -249,9 +255,17 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
         if (threadIdx.x < a.C) {
             const int64_t j = row * a.C + threadIdx.x;
             const float w = a.weight[j];
-            const float2 mz = a.mz[j];
-            f_s[threadIdx.x] = (w > 0.0f && mz.y > 0.0f) ? w / mz.y : 0.0f;
-            m_s[threadIdx.x] = mz.x;
+            // the key range was split into chunks: merge their (max, sum)
+            const float2 *mzj = a.mz + j * a.nchunk;
+            float m = kNegInf;
+            for (int c = 0; c < a.nchunk; ++c) m = fmaxf(m, mzj[c].x);
+            float z = 0.0f;
+            for (int c = 0; c < a.nchunk; ++c) {
+                const float2 q = mzj[c];
+                if (q.x != kNegInf) z += q.y * ex2_approx(q.x - m);
+            }
+            f_s[threadIdx.x] = (w > 0.0f && z > 0.0f) ? w / z : 0.0f;
+            m_s[threadIdx.x] = m;
         }
         __syncthreads();
         float *prow = a.p + row * (int64_t)a.nK;
@@ -310,7 +324,7 @@ cudaError_t launch_score_t(const ScoreArgs &a, const ScoreMaps &maps, cudaStream
     cudaError_t e = cudaFuncSetAttribute(score_mass_kernel<D, BK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.MC + 127) / 128, a.heads);
+    dim3 grid((a.MC + 127) / 128, a.heads, a.nchunk);
     score_mass_kernel<D, BK><<<grid, kScoreThreads, smem, stream>>>(maps, a);
     return cudaGetLastError();
 }
