@@ -17,7 +17,7 @@ struct KmeansArgs {
     float *cent_out;         // optional [rows][C][D]
     int32_t *sizes_out;      // optional [rows][C]
 };
-size_t kmeans_smem_bytes(int D);
+size_t kmeans_smem_bytes(int D, int C);
 cudaError_t launch_kmeans(const KmeansArgs &a, int num_sms, cudaStream_t stream);
 
 // ---- IBCS part 2: centroid . key softmax mass per key block -----------------

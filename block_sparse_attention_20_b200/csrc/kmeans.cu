@@ -11,10 +11,11 @@
 //     about 16 significant bits of the centroid; warp w takes rows
 //     32w..32w+31; the argmin (ties to the lower index) is reduced across the
 //     four lanes that share a row;
-//   - update: a stable counting sort of the rows by cluster (warp ballots),
-//     then thread x sums dimension x of each cluster's rows as four
-//     interleaved partial sums in ascending row order, combined in a fixed
-//     order (deterministic), centroid = sum / size.
+//   - update: cluster sizes from warp ballots; the per-cluster sums of the
+//     rows are one more tensor-core product, onehot(assignment)^T . Q
+//     (16 x 128 times 128 x D, exact products, fp32 accumulation in the
+//     hardware's fixed order, so the result is deterministic); centroid =
+//     sum / size.
 //
 // Rules (open in the abstract, fixed here): C_eff = min(C, n) clusters;
 // centroid j starts at row floor(j*n/C_eff); squared Euclidean distance,
@@ -43,25 +44,36 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// four 8x8 b16 matrices, transposed on the way: lane l supplies the address
+// of row l%8 of matrix l/8
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void *row_addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row_addr)));
+}
+
+// bf16 pair (lo, hi) of two 0/1 flags
+__device__ __forceinline__ uint32_t onehot_pair(bool lo, bool hi) {
+    return (lo ? 0x3F80u : 0u) | (hi ? 0x3F800000u : 0u);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a) {
     constexpr int LDQ = D + 8;  // bf16 row stride: 4*row + column-pair spreads the banks
+    const int C = a.C;
+    const int CP = C <= 8 ? 8 : 16;  // centroid rows held (one or two 8-wide MMA tiles)
     extern __shared__ __align__(16) unsigned char km_smem[];
     __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(km_smem);             // [128][LDQ]
-    float *cent = reinterpret_cast<float *>(km_smem + 128 * LDQ * 2);            // [kMaxC][D]
-    __nv_bfloat16 *chi = reinterpret_cast<__nv_bfloat16 *>(cent + kMaxC * D);    // [kMaxC][LDQ]
-    __nv_bfloat16 *clo = chi + kMaxC * LDQ;                                      // [kMaxC][LDQ]
+    float *cent = reinterpret_cast<float *>(km_smem + 128 * LDQ * 2);            // [CP][D]
+    __nv_bfloat16 *chi = reinterpret_cast<__nv_bfloat16 *>(cent + CP * D);       // [CP][LDQ]
+    __nv_bfloat16 *clo = chi + CP * LDQ;                                         // [CP][LDQ]
     __shared__ float cnorm[kMaxC];
     __shared__ int assign_s[128];
-    __shared__ int order_s[128];
-    __shared__ uint32_t mask_s[4][kMaxC];
+    __shared__ int wcnt_s[4][kMaxC];
     __shared__ int cnt_s[kMaxC];
-    __shared__ int base_s[kMaxC];
-    __shared__ int woff_s[4][kMaxC];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, cq = lane & 3;  // mma fragment coordinates
-    const int C = a.C;
     const uint32_t *qw = reinterpret_cast<const uint32_t *>(qs);
     const uint32_t *hw = reinterpret_cast<const uint32_t *>(chi);
     const uint32_t *lw = reinterpret_cast<const uint32_t *>(clo);
@@ -74,15 +86,20 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         const int ce = min(C, n);
         const __nv_bfloat16 *qblk = a.Q + (bh * (int64_t)a.N + (int64_t)i * 128) * D;
 
-        // the block's queries, row r by thread r; missing rows are zero
+        // the block's queries (contiguous in memory: coalesced 16-byte chunks);
+        // missing rows are zero
         {
-            const uint4 *src = reinterpret_cast<const uint4 *>(qblk + (int64_t)tid * D);
-            uint4 *dst = reinterpret_cast<uint4 *>(qs + tid * LDQ);
+            constexpr int CPR = D / 8;  // 16-byte chunks per row
+            const uint4 *src = reinterpret_cast<const uint4 *>(qblk);
 #pragma unroll 4
-            for (int v = 0; v < D / 8; ++v) dst[v] = tid < n ? src[v] : make_uint4(0, 0, 0, 0);
+            for (int c = tid; c < 128 * CPR; c += kKmThreads) {
+                const int r = c / CPR, x8 = c % CPR;
+                *reinterpret_cast<uint4 *>(qs + r * LDQ + x8 * 8) =
+                    r < n ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            }
         }
         __syncthreads();
-        for (int e = tid; e < kMaxC * D; e += kKmThreads) {
+        for (int e = tid; e < CP * D; e += kKmThreads) {
             const int j = e / D, x = e % D;
             cent[e] = j < ce ? __bfloat162float(qs[(int)(((int64_t)j * n) / ce) * LDQ + x]) : 0.0f;
         }
@@ -91,7 +108,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         const int rounds = a.iters > 0 ? a.iters : 1;
         for (int it = 0; it < rounds; ++it) {
             // ---- centroid operands: bf16 hi + lo, squared norms ----
-            for (int e = tid; e < kMaxC * D; e += kKmThreads) {
+            for (int e = tid; e < CP * D; e += kKmThreads) {
                 const int j = e / D, x = e % D;
                 const float c = cent[e];
                 const __nv_bfloat16 h = __float2bfloat16_rn(c);
@@ -99,7 +116,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                 clo[j * LDQ + x] = __float2bfloat16_rn(c - __bfloat162float(h));
             }
             // squared norms: warp w takes centroids w, w+4, ...; lanes split the dimensions
-            for (int j = warp; j < kMaxC; j += 4) {
+            for (int j = warp; j < CP; j += 4) {
                 float s = 0.0f;
 #pragma unroll
                 for (int x = lane; x < D; x += 32) s = fmaf(cent[j * D + x], cent[j * D + x], s);
@@ -111,13 +128,13 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
 
             // ---- assignment: q.c on tensor cores, argmin over centroids ----
             const int nt = (ce + 7) >> 3;  // 8-wide centroid tiles
-            float bestd[2][2];
-            int besti[2][2];
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const int r0 = warp * 32 + m * 16;
+                float bestd[2];
+                int besti[2];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) { bestd[m][h] = __int_as_float(0x7f800000); besti[m][h] = 0; }
+                for (int h = 0; h < 2; ++h) { bestd[h] = __int_as_float(0x7f800000); besti[h] = 0; }
                 for (int t = 0; t < nt; ++t) {
                     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -140,7 +157,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                             const int j = t * 8 + 2 * cq + u;
                             const float dj = j < ce ? fmaf(-2.0f, acc[2 * h + u], cnorm[j])
                                                     : __int_as_float(0x7f800000);
-                            if (dj < bestd[m][h]) { bestd[m][h] = dj; besti[m][h] = j; }
+                            if (dj < bestd[h]) { bestd[h] = dj; besti[h] = j; }
                         }
                 }
                 // combine the four lanes of each row (ties to the lower index)
@@ -148,66 +165,79 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int o = 1; o < 4; o <<= 1) {
-                        const float od = __shfl_xor_sync(0xffffffffu, bestd[m][h], o);
-                        const int oi = __shfl_xor_sync(0xffffffffu, besti[m][h], o);
-                        if (od < bestd[m][h] || (od == bestd[m][h] && oi < besti[m][h])) {
-                            bestd[m][h] = od;
-                            besti[m][h] = oi;
+                        const float od = __shfl_xor_sync(0xffffffffu, bestd[h], o);
+                        const int oi = __shfl_xor_sync(0xffffffffu, besti[h], o);
+                        if (od < bestd[h] || (od == bestd[h] && oi < besti[h])) {
+                            bestd[h] = od;
+                            besti[h] = oi;
                         }
                     }
                 if (cq == 0) {
-                    assign_s[r0 + g] = (r0 + g) < n ? besti[m][0] : -1;
-                    assign_s[r0 + g + 8] = (r0 + g + 8) < n ? besti[m][1] : -1;
+                    assign_s[r0 + g] = (r0 + g) < n ? besti[0] : -1;
+                    assign_s[r0 + g + 8] = (r0 + g + 8) < n ? besti[1] : -1;
                 }
             }
             __syncthreads();
-            const int best = assign_s[tid];
 
-            // ---- stable counting sort of rows by cluster ----
-            for (int j = 0; j < ce; ++j) {
-                const uint32_t m = __ballot_sync(0xffffffffu, best == j);
-                if (lane == 0) mask_s[warp][j] = m;
-            }
-            __syncthreads();
-            if (tid == 0) {
-                int acc = 0;
+            // ---- cluster sizes: ballots of this warp's rows, summed over warps ----
+            {
+                const int best = assign_s[tid];
                 for (int j = 0; j < ce; ++j) {
-                    base_s[j] = acc;
-                    for (int w = 0; w < 4; ++w) {
-                        woff_s[w][j] = acc - base_s[j];
-                        acc += __popc(mask_s[w][j]);
-                    }
-                    cnt_s[j] = acc - base_s[j];
+                    const uint32_t m = __ballot_sync(0xffffffffu, best == j);
+                    if (lane == 0) wcnt_s[warp][j] = __popc(m);
                 }
             }
             __syncthreads();
-            if (best >= 0) {
-                const int pos = base_s[best] + woff_s[warp][best] +
-                                __popc(mask_s[warp][best] & ((1u << lane) - 1u));
-                order_s[pos] = tid;
-            }
+            if (tid < ce) cnt_s[tid] = wcnt_s[0][tid] + wcnt_s[1][tid] + wcnt_s[2][tid] + wcnt_s[3][tid];
             __syncthreads();
             if (a.iters == 0) break;  // sizes from the seeds, no update
-            // ---- update: thread x sums dimension x of every cluster ----
-            for (int x = tid; x < D; x += kKmThreads) {
-                for (int j = 0; j < ce; ++j) {
-                    const int c = cnt_s[j];
-                    if (c == 0) continue;
-                    // four interleaved partial sums (rows e = 0,4,8,.. / 1,5,9,.. / ...)
-                    // in ascending row order each, combined in a fixed order
-                    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-                    const int b0 = base_s[j];
-                    int e = 0;
-                    for (; e + 4 <= c; e += 4) {
-                        s0 += __bfloat162float(qs[order_s[b0 + e] * LDQ + x]);
-                        s1 += __bfloat162float(qs[order_s[b0 + e + 1] * LDQ + x]);
-                        s2 += __bfloat162float(qs[order_s[b0 + e + 2] * LDQ + x]);
-                        s3 += __bfloat162float(qs[order_s[b0 + e + 3] * LDQ + x]);
+
+            // ---- update: sums = onehot^T (16 x 128) . Q (128 x D) ----
+            // A rows are the clusters (up to 16: one MMA tile), A columns the
+            // block's rows (1 where the row is assigned to the cluster); warp w
+            // takes the column tiles of dimensions [w*D/4, (w+1)*D/4)
+            {
+                constexpr int NT = D / 32;  // 8-wide column tiles per warp
+                float acc[NT][4];
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) acc[t][u] = 0.0f;
+                const int n0w = warp * NT * 8;
+#pragma unroll 2
+                for (int k0 = 0; k0 < 128; k0 += 16) {
+                    const int q0 = assign_s[k0 + 2 * cq], q1 = assign_s[k0 + 2 * cq + 1];
+                    const int q8 = assign_s[k0 + 2 * cq + 8], q9 = assign_s[k0 + 2 * cq + 9];
+                    uint32_t af[4];
+                    af[0] = onehot_pair(q0 == g, q1 == g);
+                    af[1] = onehot_pair(q0 == g + 8, q1 == g + 8);
+                    af[2] = onehot_pair(q8 == g, q9 == g);
+                    af[3] = onehot_pair(q8 == g + 8, q9 == g + 8);
+#pragma unroll
+                    for (int t = 0; t < NT; t += 2) {
+                        // matrices: rows k0..k0+7 / k0+8..k0+15 of column tiles t, t+1
+                        const int mi = lane >> 3;
+                        const __nv_bfloat16 *ra =
+                            qs + (k0 + (mi & 1) * 8 + (lane & 7)) * LDQ + n0w + (t + (mi >> 1)) * 8;
+                        uint32_t b[4];
+                        ldsm_x4_trans(b, ra);
+                        mma_bf16_16816(acc[t], af, b[0], b[1]);
+                        mma_bf16_16816(acc[t + 1], af, b[2], b[3]);
                     }
-                    if (e < c) s0 += __bfloat162float(qs[order_s[b0 + e] * LDQ + x]);
-                    if (e + 1 < c) s1 += __bfloat162float(qs[order_s[b0 + e + 1] * LDQ + x]);
-                    if (e + 2 < c) s2 += __bfloat162float(qs[order_s[b0 + e + 2] * LDQ + x]);
-                    cent[j * D + x] = ((s0 + s1) + (s2 + s3)) / (float)c;
+                }
+                // acc[t]: [0..1] cluster g, dimensions n0w+8t+2cq+{0,1}; [2..3] cluster g+8
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = g + 8 * h;
+                    if (j >= ce) continue;
+                    const int c = cnt_s[j];
+                    if (c == 0) continue;  // an empty cluster keeps its centroid
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        const int x = n0w + 8 * t + 2 * cq;
+                        cent[j * D + x] = acc[t][2 * h] / (float)c;
+                        cent[j * D + x + 1] = acc[t][2 * h + 1] / (float)c;
+                    }
                 }
             }
             __syncthreads();
@@ -237,30 +267,33 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
 
 }  // namespace
 
-size_t kmeans_smem_bytes(int D) {
-    const int ldq = D + 8;
-    return (size_t)128 * ldq * 2 + sizeof(float) * kMaxC * D + 2 * (size_t)kMaxC * ldq * 2;
+size_t kmeans_smem_bytes(int D, int C) {
+    const int ldq = D + 8, cp = C <= 8 ? 8 : 16;
+    return (size_t)128 * ldq * 2 + sizeof(float) * cp * D + 2 * (size_t)cp * ldq * 2;
+}
+
+template <int D>
+cudaError_t launch_kmeans_d(const KmeansArgs &a, int num_sms, cudaStream_t stream) {
+    const size_t smem = kmeans_smem_bytes(D, a.C);
+    cudaError_t e = cudaFuncSetAttribute(kmeans_qblock_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kmeans_qblock_kernel<D>, kKmThreads,
+                                                      smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = a.rows;
+    const int64_t cap = (int64_t)num_sms * per_sm;  // every CTA resident: an even share each
+    if (grid > cap) grid = cap;
+    kmeans_qblock_kernel<D><<<(unsigned)grid, kKmThreads, smem, stream>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_kmeans(const KmeansArgs &a, int num_sms, cudaStream_t stream) {
-    int64_t grid = a.rows;
-    const int64_t cap = (int64_t)num_sms * 8;
-    if (grid > cap) grid = cap;
-    if (grid < 1) return cudaSuccess;
-    const size_t smem = kmeans_smem_bytes(a.D);
-    cudaError_t e;
-    if (a.D == 128) {
-        e = cudaFuncSetAttribute(kmeans_qblock_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kmeans_qblock_kernel<128><<<(unsigned)grid, kKmThreads, smem, stream>>>(a);
-    } else {
-        e = cudaFuncSetAttribute(kmeans_qblock_kernel<64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kmeans_qblock_kernel<64><<<(unsigned)grid, kKmThreads, smem, stream>>>(a);
-    }
-    return cudaGetLastError();
+    if (a.rows < 1) return cudaSuccess;
+    return a.D == 128 ? launch_kmeans_d<128>(a, num_sms, stream)
+                      : launch_kmeans_d<64>(a, num_sms, stream);
 }
 
 }  // namespace abatt
