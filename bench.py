@@ -258,24 +258,15 @@ def main():
     c = counts.cpu().numpy().astype(np.int64)
     idx_h = idx.cpu().numpy()
     bpt = 128 // w.Bk
-    # executed tiles: each pair of neighbouring query blocks of a head runs
-    # both rows over the union of their two lists
-    tiles = 0
+    # executed tiles: every row runs its own drawn blocks, 128/Bk per tile
+    # (pairs of neighbouring rows share the gathers of common tiles, not the math)
     last = w.nK - 1
     tail = w.N - last * w.Bk
     keys = np.zeros(rows, dtype=np.int64)
     for r in range(rows):
         L = c[r]
         keys[r] = L * w.Bk - (w.Bk - tail if L and idx_h[r, :L][-1] == last else 0)
-    for hd in range(w.B * w.H):
-        for j in range(0, w.nQ, 2):
-            r0 = hd * w.nQ + j
-            u = set(idx_h[r0, :c[r0]].tolist())
-            n_rows = 1
-            if j + 1 < w.nQ:
-                u |= set(idx_h[r0 + 1, :c[r0 + 1]].tolist())
-                n_rows = 2
-            tiles += n_rows * ((len(u) + bpt - 1) // bpt)
+    tiles = int(((c + bpt - 1) // bpt).sum())
     exec_flop = tiles * 4.0 * 128 * 128 * w.d
     # algorithmic work: valid query rows x valid drawn keys
     nrows_q = np.minimum(128, w.N - (np.arange(rows) % w.nQ) * 128)
@@ -309,7 +300,7 @@ def main():
                      "kernel": "gather_attn_kernel", "flops": "algorithmic (valid query rows x drawn keys)",
                      "peak_source": f"{src} bf16 sustained"},
         "device_status": status,
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": 7 * args.steps,
         "clocks": clk.summary(),
     }
 

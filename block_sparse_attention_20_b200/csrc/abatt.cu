@@ -73,8 +73,8 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
 
 // ---- workspace layout ----------------------------------------------------------
 struct Layout {
-    size_t hdr, cent_hi, cent_lo, weight, r, mref, mz;  // select
-    size_t ulen, ublk, ulw;                               // attention (pair unions)
+    size_t hdr, cent16, k16, weight, r, mref, mz;  // select
+    size_t useg, ublk, ulw;                               // attention (pair segments)
     size_t p, counts, idx, logw;                          // forward
     size_t total;
 };
@@ -89,8 +89,8 @@ Layout layout(abatt_call call, const Geom &g) {
     off += sizeof(WsHeader);
     if (call == ABATT_CALL_SELECT || call == ABATT_CALL_FORWARD) {
         const size_t crow = (size_t)g.rows * g.C;
-        L.cent_hi = off; off = align256(off + crow * g.d * 2);
-        L.cent_lo = off; off = align256(off + crow * g.d * 2);
+        L.cent16 = off;  off = align256(off + crow * g.d * 2);
+        L.k16 = off;     off = align256(off + (size_t)g.heads * g.N * g.d * 2);
         L.weight = off;  off = align256(off + crow * 4);
         L.r = off;       off = align256(off + crow * g.ldr * 4);
         L.mref = off;    off = align256(off + crow * g.nT * 4);
@@ -98,7 +98,7 @@ Layout layout(abatt_call call, const Geom &g) {
     }
     if (call == ABATT_CALL_ATTENTION || call == ABATT_CALL_FORWARD) {
         const size_t pairs = (size_t)pairs_of(g);
-        L.ulen = off; off = align256(off + pairs * 4);
+        L.useg = off; off = align256(off + pairs * 16);
         L.ublk = off; off = align256(off + pairs * g.nK * 4);
         L.ulw = off;  off = align256(off + pairs * 2 * g.nK * 4);
     }
@@ -150,16 +150,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D bf16 map over [outer][rows][d] with a (64, box_rows, 1) box, 128-byte
-// swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t outer, int box_rows) {
+// 3-D map of 16-bit elements (bf16 unless stated) over [outer][rows][d] with
+// a (64, box_rows, 1) box, 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t outer, int box_rows,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)outer};
     const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+    return fn(m, dtype, 3, const_cast<void *>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -199,23 +200,25 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     ka.Q = static_cast<const __nv_bfloat16 *>(Q);
     ka.rows = g.rows; ka.nQ = g.nQ; ka.N = g.N; ka.D = g.d; ka.C = g.C; ka.iters = g.I;
     ka.logit_mul = cfg->scale * kLog2eF;
-    ka.cent_hi = at<__nv_bfloat16>(ws, L.cent_hi);
-    ka.cent_lo = at<__nv_bfloat16>(ws, L.cent_lo);
+    ka.cent16 = at<__half>(ws, L.cent16);
     ka.weight = at<float>(ws, L.weight);
     ka.cent_out = cent_out;
     ka.sizes_out = sizes_out;
     cudaError_t e = launch_kmeans(ka, sms, st);
     if (e != cudaSuccess) return ABATT_ERR_CUDA;
 
+    __half *k16 = at<__half>(ws, L.k16);
+    e = launch_keys_f16(static_cast<const __nv_bfloat16 *>(K), k16, g.heads * g.N * g.d / 8, sms, st);
+    if (e != cudaSuccess) return ABATT_ERR_CUDA;
+
     ScoreMaps sm;
     const int64_t MC = (int64_t)g.nQ * g.C;
-    if (!make_map(&sm.a_hi, ka.cent_hi, g.d, MC, g.heads, 128) ||
-        !make_map(&sm.a_lo, ka.cent_lo, g.d, MC, g.heads, 128) ||
-        !make_map(&sm.k, K, g.d, g.N, g.heads, 128))
+    if (!make_map(&sm.a, ka.cent16, g.d, MC, g.heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_map(&sm.k, k16, g.d, g.N, g.heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return ABATT_ERR_CUDA;
     ScoreArgs sa;
     sa.heads = (int)g.heads; sa.N = g.N; sa.D = g.d; sa.Bk = g.Bk; sa.MC = (int)MC;
-    sa.nT = g.nT; sa.ldr = g.ldr; sa.use_lo = 1;
+    sa.nT = g.nT; sa.ldr = g.ldr;
     score_chunks(g.nT, ((int)MC + 127) / 128 * g.heads, sms, &sa.nchunk, &sa.chunk_tiles);
     sa.r = at<float>(ws, L.r);
     sa.mref = at<float>(ws, L.mref);
@@ -253,7 +256,7 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     PairArgs pa;
     pa.rows = g.rows; pa.pairs = pairs_of(g); pa.nQ = g.nQ; pa.nK = g.nK; pa.capacity = capacity; pa.cap_u = g.nK;
     pa.counts = counts; pa.idx = idx; pa.logw = logw;
-    pa.ulen = at<int32_t>(ws, L.ulen);
+    pa.useg = at<int32_t>(ws, L.useg);
     pa.ublk = at<int32_t>(ws, L.ublk);
     pa.ulw = at<float>(ws, L.ulw);
     pa.status = &hdr->status;
@@ -281,7 +284,7 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     a.rows = g.rows; a.pairs = pairs_of(g); a.nQ = g.nQ; a.N = g.N; a.D = g.d; a.Bk = g.Bk;
     a.nK = g.nK; a.cap_u = g.nK; a.k_fold = fold ? 1 : 0;
     a.scale_log2 = cfg->scale * kLog2eF;
-    a.ulen = pa.ulen; a.ublk = pa.ublk; a.ulw = pa.ulw;
+    a.useg = pa.useg; a.ublk = pa.ublk; a.ulw = pa.ulw;
     a.O = static_cast<__nv_bfloat16 *>(O);
     a.lse = lse;
     a.hdr = hdr;

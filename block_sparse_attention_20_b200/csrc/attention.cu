@@ -46,6 +46,12 @@ constexpr int kAttnThreads = 576;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
+// exponent pairs of every eight that the softmax evaluates with the FMA-pipe
+// polynomial (the others use ex2); balances the two pipes
+#ifndef ABATT_ATTN_POLY_OF_8
+#define ABATT_ATTN_POLY_OF_8 3
+#endif
+constexpr int kAttnPolyOf8 = ABATT_ATTN_POLY_OF_8;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -64,12 +70,14 @@ __device__ __forceinline__ bool union_entry_ok(const int32_t *idx, int j, int k,
 }
 
 __global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArgs a) {
-    // [W] membership bitmap of each row, [W] union prefix (exclusive) per word
+    // [W] membership bitmap of each row, then per word the exclusive prefix of
+    // the three segment counts (both rows, row 0 only, row 1 only)
     extern __shared__ uint32_t sm_union[];
-    __shared__ int32_t wsum[kUnionThreads / 32];
+    __shared__ uint64_t wsum[kUnionThreads / 32];
     const int W = (a.nK + 31) >> 5;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t *bA = sm_union, *bB = sm_union + W, *pre = sm_union + 2 * W;
+    uint32_t *bA = sm_union, *bB = sm_union + W;
+    uint32_t *preB = sm_union + 2 * W, *preA = preB + W, *preC = preA + W;
     for (int64_t pr = blockIdx.x; pr < a.pairs; pr += gridDim.x) {
         __syncthreads();
         for (int w = tid; w < 2 * W; w += kUnionThreads) sm_union[w] = 0;
@@ -89,61 +97,77 @@ __global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArg
             }
         }
         if (__syncthreads_or(bad) && tid == 0) raise_flag(a.status, ABATT_DEVFLAG_BADLIST);
-        // exclusive prefix of the union's popcount per word: each thread owns a
-        // contiguous run of words, block-wide scan of the run totals
+        // exclusive prefix of the three popcounts per word, packed 21 bits
+        // each into one 64-bit scan: each thread owns a contiguous run of words
         const int per = (W + kUnionThreads - 1) / kUnionThreads;
         const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
-        int cnt = 0;
-        for (int w = w0; w < w1; ++w) cnt += __popc(bA[w] | bB[w]);
-        int x = cnt;
+        auto counts3 = [&](int w) -> uint64_t {
+            const uint32_t x = bA[w], y = bB[w];
+            return (uint64_t)__popc(x & y) | ((uint64_t)__popc(x & ~y) << 21) |
+                   ((uint64_t)__popc(y & ~x) << 42);
+        };
+        uint64_t cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += counts3(w);
+        uint64_t x = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
         if (lane == 31) wsum[warp] = x;
         __syncthreads();
-        int run = x - cnt, total = 0;
+        uint64_t run = x - cnt, total = 0;
         for (int w = 0; w < kUnionThreads / 32; ++w) {
             if (w < warp) run += wsum[w];
             total += wsum[w];
         }
+        constexpr uint64_t kM21 = (1u << 21) - 1u;
         for (int w = w0; w < w1; ++w) {
-            pre[w] = run;
-            run += __popc(bA[w] | bB[w]);
+            preB[w] = (uint32_t)(run & kM21);
+            preA[w] = (uint32_t)((run >> 21) & kM21);
+            preC[w] = (uint32_t)(run >> 42);
+            run += counts3(w);
         }
+        const int nb = (int)(total & kM21), na = (int)((total >> 21) & kM21), nc = (int)(total >> 42);
         __syncthreads();
         int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
-        float *uw = a.ulw + pr * 2 * (int64_t)a.cap_u;
-        // union block ids in ascending order; both log-weights start as "not drawn"
+        // union layout: [both rows | row 0 only | row 1 only], each ascending
         for (int w = tid; w < W; w += kUnionThreads) {
-            uint32_t mu = bA[w] | bB[w];
-            int pos = pre[w];
-            while (mu) {
-                const int bit = __ffs(mu) - 1;
-                mu &= mu - 1;
-                if (pos < a.cap_u) {
-                    ub[pos] = w * 32 + bit;
-                    uw[pos] = -1.0f;
-                    uw[a.cap_u + pos] = -1.0f;
+            const uint32_t xa = bA[w], xb = bB[w];
+            const uint32_t seg[3] = {xa & xb, xa & ~xb, xb & ~xa};
+            const int base[3] = {(int)preB[w], nb + (int)preA[w], nb + na + (int)preC[w]};
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                int pos = base[q];
+                for (uint32_t mu = seg[q]; mu; mu &= mu - 1) {
+                    if (pos < a.cap_u) ub[pos] = w * 32 + __ffs(mu) - 1;
+                    ++pos;
                 }
-                ++pos;
             }
         }
-        __syncthreads();
-        // each valid drawn entry writes its log-weight at its union position
+        // each valid drawn entry writes its row's log-weight at its position
+        float *uw = a.ulw + pr * 2 * (int64_t)a.cap_u;
         for (int s = 0; s < 2; ++s) {
             const int32_t *idx = a.idx + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
             const float *lw = a.logw + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
             for (int j = tid; j < L[s]; j += kUnionThreads) {
                 const int k = idx[j];
                 if (!union_entry_ok(idx, j, k, a.nK)) continue;
-                const uint32_t mu = bA[k >> 5] | bB[k >> 5];
-                const int pos = pre[k >> 5] + __popc(mu & ((1u << (k & 31)) - 1u));
+                const int w = k >> 5;
+                const uint32_t below = (1u << (k & 31)) - 1u;
+                const uint32_t xa = bA[w], xb = bB[w];
+                int pos;
+                if ((xa & xb) >> (k & 31) & 1u) pos = (int)preB[w] + __popc(xa & xb & below);
+                else if (s == 0) pos = nb + (int)preA[w] + __popc(xa & ~xb & below);
+                else pos = nb + na + (int)preC[w] + __popc(xb & ~xa & below);
                 if (pos < a.cap_u) uw[s * a.cap_u + pos] = lw[j];
             }
         }
-        if (tid == 0) a.ulen[pr] = min(total, a.cap_u);
+        if (tid == 0) {
+            a.useg[pr * 4 + 0] = nb;
+            a.useg[pr * 4 + 1] = na;
+            a.useg[pr * 4 + 2] = nc;
+        }
     }
 }
 
@@ -152,8 +176,49 @@ template <int D>
 struct AttnCfg {
     static constexpr int CH = D / 64;
     static constexpr uint32_t TILE = 128u * D * 2u;
-    static constexpr int ST = D == 128 ? 4 : 9;  // K/V ring stages
+    static constexpr int ST = D == 128 ? 5 : 12;  // K/V ring stages (Q tiles + ring <= 225 KB)
     static constexpr size_t SMEM = (size_t)(2 + ST) * TILE + 1024;
+};
+
+// The tile schedule of one pair.  Row s walks its sequence (row 0: [both |
+// row 0 only], row 1: [both | row 1 only]) in tiles of BPT blocks: n[s]
+// tiles.  The first tb tiles lie wholly inside the shared segment and are
+// gathered once for both rows; later tiles are gathered per row.  Gathers
+// ("groups", a K tile and a V tile each, ring slots 2g and 2g+1 after the
+// pair's first slot) run in step order: shared tiles 0..tb-1, then for each
+// step t >= tb row 0's tile (if t < n[0]) and row 1's tile (if t < n[1]).
+struct PairPlan {
+    int nb, na, L0, L1, n0, n1, tb, m, groups;
+    __device__ __forceinline__ PairPlan(const int32_t *useg, int64_t pr, bool has1, int bpt) {
+        nb = useg[pr * 4 + 0];
+        na = useg[pr * 4 + 1];
+        const int nc = useg[pr * 4 + 2];
+        L0 = nb + na;
+        L1 = has1 ? nb + nc : 0;
+        n0 = (L0 + bpt - 1) / bpt;
+        n1 = (L1 + bpt - 1) / bpt;
+        tb = has1 ? nb / bpt : 0;
+        m = max(0, min(n0, n1) - tb);
+        groups = n0 + n1 - tb;
+    }
+    __device__ __forceinline__ int L(int s) const { return s ? L1 : L0; }
+    __device__ __forceinline__ int n(int s) const { return s ? n1 : n0; }
+    // gather group of row s's tile t
+    __device__ __forceinline__ int group(int s, int t) const {
+        if (t < tb) return t;
+        const int d = t - tb;
+        return d < m ? tb + 2 * d + s : tb + 2 * m + (d - m);
+    }
+    // row (-1: shared) and tile of gather group g
+    __device__ __forceinline__ void tile_of(int g, int *s, int *t) const {
+        if (g < tb) { *s = -1; *t = g; return; }
+        const int r = g - tb;
+        if (r < 2 * m) { *s = r & 1; *t = tb + (r >> 1); return; }
+        *s = n0 > n1 ? 0 : 1;
+        *t = tb + m + (r - 2 * m);
+    }
+    // entry e of row s's sequence -> position in the pair's block array
+    __device__ __forceinline__ int pos(int s, int e) const { return (s == 0 || e < nb) ? e : e + na; }
 };
 
 template <int D, int BK, bool KFOLD>
@@ -226,18 +291,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t rp = 0;
         bool ok = true;
         for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
-            const int U = a.ulen[pr];
-            const int n = (U + BPT - 1) / BPT;
-            if (n == 0) continue;
             int64_t rr[2];
             pair_rows(pr, a.nQ, &rr[0], &rr[1]);
+            const PairPlan P(a.useg, pr, rr[1] >= 0, BPT);
+            if (P.groups == 0) continue;
             const int hd = (int)(rr[0] / a.nQ);
             const int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
-            int nxt = (lane < BPT && lane < U) ? __ldg(ub + lane) : -1;
+            // block index of this lane in gather group g (-1: empty slot)
+            auto blk_of = [&](int g) -> int {
+                if (g >= P.groups || lane >= BPT) return -1;
+                int s, t;
+                P.tile_of(g, &s, &t);
+                const int sr = s < 0 ? 0 : s, e = t * BPT + lane;
+                return e < P.L(sr) ? __ldg(ub + P.pos(sr, e)) : -1;
+            };
+            int nxt = blk_of(0);
             if (lane == 0) {
                 for (int s = 0; s < 2; ++s) {
                     const int64_t row = rr[s];
-                    if (row < 0) continue;
+                    if (row < 0 || P.n(s) == 0) continue;
                     if (q_loads[s] > 0 && !mbar_wait(&bar_qe[s], (q_loads[s] - 1) & 1, wc, 0x202)) {
                         ok = false;
                         break;
@@ -250,11 +322,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            for (int t = 0; ok && t < n; ++t) {
+            for (int g = 0; ok && g < P.groups; ++g) {
                 const int blk = nxt;
-                const int jn = (t + 1) * BPT + lane;
-                nxt = (lane < BPT && jn < U) ? __ldg(ub + jn) : -1;
-                for (int kv = 0; kv < 2; ++kv) {  // K(t) then V(t)
+                nxt = blk_of(g + 1);
+                for (int kv = 0; kv < 2; ++kv) {  // K then V of the group
                     const int stg = rp % ST;
                     if (lane == 0) {
                         if (rp >= ST && !mbar_wait(&bar_kve[stg], ((rp / ST) - 1) & 1, wc, 0x201)) ok = false;
@@ -268,8 +339,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         if (kv == 0) {
                             if (KFOLD) {
                                 // groups of 8 rows with all heads folded: a box of Bk/8 groups
-                                const int g = valid ? hd * groups_per_head + blk * (BK / 8) : 0x7fffff00;
-                                tma_load_4d(dst + lane * BLK, &maps.k, &bar_kvf[stg], 0, 0, 0, g);
+                                const int gi = valid ? hd * groups_per_head + blk * (BK / 8) : 0x7fffff00;
+                                tma_load_4d(dst + lane * BLK, &maps.k, &bar_kvf[stg], 0, 0, 0, gi);
                             } else {
                                 const int y = valid ? blk * BK : a.nK * BK;
                                 for (int c = 0; c < CH; ++c)
@@ -316,7 +387,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
                 const uint32_t koff =
                     KFOLD ? (kk >> 2) * 1024 + (kk & 3) * 32 : (kk >> 2) * 16384 + (kk & 3) * 32;
-                umma_bf16_ss_w(tmem + s * 128, qd + (qoff >> 4), kd + (koff >> 4), idesc_s, kk > 0);
+                umma_ss_w(tmem + s * 128, qd + (qoff >> 4), kd + (koff >> 4), idesc_s, kk > 0);
             }
             if (release) umma_commit_w(&bar_kve[stg]);
             umma_commit_w(&bar_sf[s]);
@@ -332,7 +403,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t boff = (uint32_t)((16 * j) / BK) * BLK + (uint32_t)((16 * j) % BK) * 128;
-                umma_bf16_ts_w(tmem + 256 + s * 128, tmem + s * 128 + j * 8, vd + (boff >> 4), idesc_o,
+                umma_ts_w(tmem + 256 + s * 128, tmem + s * 128 + j * 8, vd + (boff >> 4), idesc_o,
                                (t > 0 || j > 0) ? 1u : 0u);
             }
             if (release) umma_commit_w(&bar_kve[stg]);
@@ -344,37 +415,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             return true;
         };
         for (int64_t pr = blockIdx.x; ok && pr < a.pairs; pr += gridDim.x) {
-            const int U = __shfl_sync(0xffffffffu, a.ulen[pr], 0);
-            const int n = (U + BPT - 1) / BPT;
-            if (n == 0) continue;
             int64_t rr[2];
             pair_rows(pr, a.nQ, &rr[0], &rr[1]);
-            const bool has1 = rr[1] >= 0;
-            for (int s = 0; ok && s < (has1 ? 2 : 1); ++s) {
+            const PairPlan P(a.useg, pr, rr[1] >= 0, BPT);
+            if (P.groups == 0) continue;
+            for (int s = 0; ok && s < 2; ++s) {
+                if (P.n(s) == 0) continue;
                 if (!wait_all(&bar_qf[s], q_uses[s] & 1, 0x207)) ok = false;
                 ++q_uses[s];
             }
             const uint32_t base = rp;
-            // issue order: S0(0) S1(0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ...
-            // Each row's chain is softmax(t) -> PV(t) -> S(t+1) (S(t+1) overwrites
-            // the P(t) that PV(t) reads; tcgen05 MMAs of one thread run in issue
-            // order).  Waits for K/V data sit before the wait on P, so once P is
-            // ready nothing else delays the two MMAs of its row.
-            if (!wait_kv(base, 0x203)) ok = false;
-            if (ok) op_s(0, base, !has1, n == 1);
-            if (ok && has1) op_s(1, base, true, n == 1);
-            for (int t = 0; ok && t < n; ++t) {
-                const uint32_t kp = base + 2 * t, vp = kp + 1, kn = kp + 2;
-                const bool more = t + 1 < n;
-                if (!wait_kv(vp, 0x206) || (more && !wait_kv(kn, 0x203))) { ok = false; break; }
-                if (!op_pv(0, vp, t, !has1, !more)) { ok = false; break; }
-                if (more) op_s(0, kn, !has1, t + 1 == n - 1);
-                if (has1) {
-                    if (!op_pv(1, vp, t, true, !more)) { ok = false; break; }
-                    if (more) op_s(1, kn, true, t + 1 == n - 1);
+            auto kpos = [&](int s, int t) -> uint32_t { return base + 2u * (uint32_t)P.group(s, t); };
+            // a shared tile's slots are freed by row 1's MMA (issued after row 0's)
+            auto frees = [&](int s, int t) -> bool { return t >= P.tb || s == 1; };
+            // issue order per step t: PV0(t) S0(t+1) PV1(t) S1(t+1).  Each row's
+            // chain is softmax(t) -> PV(t) -> S(t+1) (S(t+1) overwrites the P(t)
+            // that PV(t) reads; tcgen05 MMAs of one thread run in issue order).
+            // Waits for K/V data sit before the wait on P, so once P is ready
+            // nothing else delays the two MMAs of its row.
+            for (int s = 0; ok && s < 2; ++s) {
+                if (P.n(s) == 0) continue;
+                if (!wait_kv(kpos(s, 0), 0x203)) { ok = false; break; }
+                op_s(s, kpos(s, 0), frees(s, 0), P.n(s) == 1);
+            }
+            const int T = max(P.n0, P.n1);
+            for (int t = 0; ok && t < T; ++t) {
+                for (int s = 0; s < 2; ++s) {
+                    if (t >= P.n(s)) continue;
+                    const bool more = t + 1 < P.n(s);
+                    const uint32_t vp = kpos(s, t) + 1;
+                    if (!wait_kv(vp, 0x206) || (more && !wait_kv(kpos(s, t + 1), 0x203))) { ok = false; break; }
+                    if (!op_pv(s, vp, t, frees(s, t), !more)) { ok = false; break; }
+                    if (more) op_s(s, kpos(s, t + 1), frees(s, t + 1), t + 2 == P.n(s));
                 }
             }
-            rp = base + 2 * n;
+            rp = base + 2u * (uint32_t)P.groups;
         }
     } else if (warp >= 2) {
         // ================================ softmax =====================================
@@ -398,8 +473,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             pair_rows(pr, a.nQ, &rr[0], &rr[1]);
             const int64_t row = rr[s];
             if (row < 0) continue;  // the pair's second row does not exist
-            const int U = a.ulen[pr];
-            const int n = (U + BPT - 1) / BPT;
+            const PairPlan P(a.useg, pr, rr[1] >= 0, BPT);
+            const int U = P.L(s), n = P.n(s);
             const int i = (int)(row % a.nQ), hd = (int)(row / a.nQ);
             const int nrows = min(128, a.N - i * 128);
             const int64_t tok = (int64_t)hd * a.N + (int64_t)i * 128 + r;
@@ -414,9 +489,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 int tail_k = -1, tail_keep = BK;
 #pragma unroll
                 for (int k = 0; k < HB; ++k) {
-                    const int j = t * BPT + (BPT >= 2 ? hh * HB + k : 0);
+                    const int e = t * BPT + (BPT >= 2 ? hh * HB + k : 0);
                     bias[k] = kNegInf;
-                    if (j < U) {
+                    if (e < U) {
+                        const int j = P.pos(s, e);
                         const float w = __ldg(lw + j);
                         if (w >= 0.0f) bias[k] = w * kLog2e;
                         const int b = __ldg(ub + j);
@@ -467,18 +543,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const float m_sub = (m_use == kNegInf) ? 0.0f : m_use;
 #pragma unroll
                 for (int k = 0; k < HB; ++k) bias[k] -= m_sub;  // now the exponent offset
-                float rs = 0.0f;
+                // exponents two at a time (packed fp32 FMA / add); a fixed share
+                // of the pairs goes to the FMA-pipe polynomial, the rest to ex2
+                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+                float2 rs2[4];  // four independent partial row sums
+#pragma unroll
+                for (int u = 0; u < 4; ++u) rs2[u] = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
+                        // columns j, j+1 lie in one key block (blocks are >= 16 wide)
                         const int k0 = BPT >= 2 ? (c * 32 + j) / BK : 0;
-                        const int k1 = BPT >= 2 ? (c * 32 + j + 1) / BK : 0;
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(v[c][j]), a.scale_log2, bias[k0]));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(v[c][j + 1]), a.scale_log2, bias[k1]));
-                        rs += p0 + p1;
-                        pk[j >> 1] = pack_bf16x2(p0, p1);
+                        const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1])),
+                                                    sc2, make_float2(bias[k0], bias[k0]));
+                        float2 p;
+                        if (((c * 16 + (j >> 1)) & 7) < kAttnPolyOf8) {
+                            p = exp2_poly2<3>(x);
+                        } else {
+                            p.x = ex2_approx(x.x);
+                            p.y = ex2_approx(x.y);
+                        }
+                        rs2[(j >> 1) & 3] = __fadd2_rn(rs2[(j >> 1) & 3], p);
+                        pk[j >> 1] = pack_bf16x2(p.x, p.y);
                     }
                     // P (bf16 pairs) over the row's S: this half's keys 64*hh + 32c + 0..31
                     // go to packed columns 32*hh + 16c + 0..15; both halves of the warp
@@ -503,7 +591,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_pf[s]);
-                l = fmaf(l, alpha, rs);
+                const float2 rs = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+                l = fmaf(l, alpha, rs.x + rs.y);
                 m_run = m_use;
             }
             if (!ok) break;
@@ -606,7 +695,7 @@ cudaError_t launch_attn_d(const AttnArgs &a, const AttnMaps &maps, int num_sms, 
 
 cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t stream) {
     if (a.pairs < 1) return cudaSuccess;
-    const size_t smem = sizeof(uint32_t) * 3 * (size_t)((a.nK + 31) / 32);
+    const size_t smem = sizeof(uint32_t) * 5 * (size_t)((a.nK + 31) / 32);
     int64_t grid = a.pairs;
     if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
     pair_union_kernel<<<(unsigned)grid, kUnionThreads, smem, stream>>>(a);

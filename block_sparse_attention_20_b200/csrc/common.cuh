@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -169,8 +170,9 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16: fp16 or bf16 operands (the
+// instruction descriptor says which), fp32 accumulate.
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -182,7 +184,7 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16: A (M x K bf16) is read from
 // tensor memory, lane m = row m, K packed two bf16 per 32-bit column.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -195,7 +197,7 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
 // Arrive on `bar` once every MMA issued so far by this thread has completed.
 // Warp-converged forms: every lane of the warp executes them (so the
 // operands stay warp-uniform) and one elected lane issues the instruction.
-__device__ __forceinline__ void umma_bf16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t"
@@ -205,7 +207,7 @@ __device__ __forceinline__ void umma_bf16_ss_w(uint32_t d_tmem, uint64_t a_desc,
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-__device__ __forceinline__ void umma_bf16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t"
@@ -335,6 +337,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major 
            | ((uint32_t)(M >> 4) << 24);     // M / 16
 }
 
+// Same for fp16 A and B (format code 0), fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4)                      // D format: f32
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm100 version bits.
 //   K-major operand: rows of 64 bf16 (128 B) in 8-row / 1024 B atoms; SBO =
 //   distance between 8-row groups.  LBO unused (1).
@@ -367,6 +376,42 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x of two values on the FMA pipe, for x <= 0, so that the special-function
+// unit (one ex2 per element, a quarter of the FMA rate) can share the
+// exponentials with the FMA units.  Cody-Waite additive reduction x = j + f,
+// j = floor(x) from a round-down add of 1.5*2^23 (the integer lands in the
+// low mantissa bits), f = x - j in [0, 1) (both exact); 2^f from a polynomial
+// with constant term 1 whose other coefficients minimise the largest relative
+// error on [0, 1] (fitted by csrc/exp2_poly_fit.py: degree 3 -> 8.6e-5,
+// degree 4 -> 2.9e-6); 2^j is added into the exponent field.  Inputs are
+// clamped at -127, where the result is exactly +0 (so a -inf logit gives 0);
+// on (-127, -126) the result is below 2^-126 but not accurate.
+template <int DEG>
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    static_assert(DEG == 3 || DEG == 4, "fitted degrees: 3, 4");
+    x.x = fmaxf(x.x, -127.0f);
+    x.y = fmaxf(x.y, -127.0f);
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
+    const float2 t = __fadd2_rd(x, magic);                          // floor(x) + 1.5*2^23
+    const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);   // x - j, exact
+    float2 p;
+    if constexpr (DEG == 3) {
+        p = __ffma2_rn(make_float2(7.706713676e-02f, 7.706713676e-02f), f,
+                       make_float2(2.276448607e-01f, 2.276448607e-01f));
+        p = __ffma2_rn(p, f, make_float2(6.951168180e-01f, 6.951168180e-01f));
+    } else {
+        p = __ffma2_rn(make_float2(1.342739072e-02f, 1.342739072e-02f), f,
+                       make_float2(5.224123225e-02f, 5.224123225e-02f));
+        p = __ffma2_rn(p, f, make_float2(2.412807941e-01f, 2.412807941e-01f));
+        p = __ffma2_rn(p, f, make_float2(6.930447817e-01f, 6.930447817e-01f));
+    }
+    p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
+    // (t's bits << 23) keeps only j's low bits: j * 2^23 modulo 2^32
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }

@@ -11,8 +11,7 @@ struct KmeansArgs {
     int64_t rows;            // B*H*nQ
     int nQ, N, D, C, iters;
     float logit_mul;         // scale * log2(e), folded into the GEMM operand
-    __nv_bfloat16 *cent_hi;  // [rows*C][D]
-    __nv_bfloat16 *cent_lo;  // [rows*C][D]
+    __half *cent16;          // [rows*C][D] scoring operand: fp16 of the scaled centroids
     float *weight;           // [rows][C]  n_j / n
     float *cent_out;         // optional [rows][C][D]
     int32_t *sizes_out;      // optional [rows][C]
@@ -31,7 +30,6 @@ struct ScoreArgs {
     int MC;        // centroid rows per head (nQ*C)
     int nT;        // key tiles per head, ceil(N/128)
     int ldr;       // row stride of r in floats (nT * 128/Bk)
-    int use_lo;    // add the lo half of the split centroids (fp32-accurate logits)
     int nchunk;    // the key tiles are split into nchunk ranges of chunk_tiles (one CTA each)
     int chunk_tiles;
     float *r;      // [heads*MC][ldr]
@@ -41,10 +39,16 @@ struct ScoreArgs {
     uint64_t wait_ns;
 };
 struct ScoreMaps {
-    CUtensorMap a_hi, a_lo, k;
+    CUtensorMap a;  // fp16 scaled centroids [heads][MC][D], box (64, 128, 1)
+    CUtensorMap k;  // fp16 keys [heads][N][D], box (64, 128, 1)
 };
 cudaError_t launch_score(const ScoreArgs &a, const ScoreMaps &maps, int num_sms,
                          cudaStream_t stream);
+
+// Keys to fp16 for the scoring GEMM (bf16 -> fp16 is exact inside fp16's
+// normal range; magnitudes beyond 65504 saturate).  n8 = elements / 8.
+cudaError_t launch_keys_f16(const __nv_bfloat16 *K, __half *K16, int64_t n8, int num_sms,
+                            cudaStream_t stream);
 
 // Combine the C centroids of each query block into p (see score.cu).
 struct CombineArgs {
@@ -74,9 +78,12 @@ cudaError_t launch_sample(const SampleArgs &a, int num_sms, cudaStream_t stream)
 // ---- gather attention -----------------------------------------------------
 // Query blocks are processed in pairs of neighbours of the same head: pair
 // (h, j) holds blocks 2j and 2j+1 of head h (the last pair of a head is a
-// single block when nQ is odd).  A pre-pass merges the pair's two ascending
-// lists into one ascending union; every union block is gathered once and
-// used by both rows, each row masking the blocks it did not draw.
+// single block when nQ is odd).  A pre-pass lays the pair's two lists out as
+// one array of three ascending segments, [blocks both rows drew | row 0 only
+// | row 1 only] (nb, na, nc entries).  Row 0 walks [both | row 0 only], row 1
+// walks [both | row 1 only]: each row runs over exactly its own blocks, and
+// the 128-key tiles that lie wholly inside the shared segment are gathered
+// once for both rows.
 __host__ __device__ __forceinline__ int64_t pairs_per_head(int nQ) { return (nQ + 1) / 2; }
 
 // Rows of pair `pr`: first row, and the second row or -1.
@@ -92,9 +99,9 @@ struct PairArgs {
     int nQ, nK, capacity, cap_u;
     const int32_t *counts, *idx;
     const float *logw;
-    int32_t *ulen;  // [pairs]
-    int32_t *ublk;  // [pairs][cap_u]   ascending union of the two lists
-    float *ulw;     // [pairs][2][cap_u] log-weight of each row, -1 = not drawn
+    int32_t *useg;  // [pairs][4]       nb, na, nc (segment lengths), unused
+    int32_t *ublk;  // [pairs][cap_u]   [both | row 0 only | row 1 only], ascending within each
+    float *ulw;     // [pairs][2][cap_u] row s's log-weight at the positions of its blocks
     uint32_t *status;
 };
 cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t stream);
@@ -105,7 +112,7 @@ struct AttnArgs {
     int cap_u;
     int k_fold;        // K tiles via head-folded 4-D boxes (needs N % 8 == 0)
     float scale_log2;  // scale * log2(e)
-    const int32_t *ulen, *ublk;
+    const int32_t *useg, *ublk;
     const float *ulw;
     __nv_bfloat16 *O;  // [B*H][N][D]
     float *lse;        // optional [B*H][N]

@@ -22,10 +22,9 @@
 // ties to the lower index; an empty cluster keeps its centroid; cluster
 // sizes come from the last round's assignment.
 //
-// Outputs: scaled centroids split into bf16 hi + lo parts (the scoring GEMM
-// operand, pre-multiplied by scale*log2(e) so the GEMM yields base-2
-// logits), the cluster weights n_j/n, and optionally the fp32 centroids and
-// cluster sizes.
+// Outputs: the centroids pre-multiplied by scale*log2(e) and rounded to fp16
+// (the scoring GEMM operand, so the GEMM yields base-2 logits), the cluster
+// weights n_j/n, and optionally the fp32 centroids and cluster sizes.
 #include "kernels.cuh"
 
 namespace abatt {
@@ -248,12 +247,8 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         for (int e = tid; e < C * D; e += kKmThreads) {
             const int j = e / D, x = e % D;
             const float c = j < ce ? cent[j * D + x] : 0.0f;
-            const float v = c * mul;
-            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
             const int64_t o = (row * C + j) * (int64_t)D + x;
-            a.cent_hi[o] = hi;
-            a.cent_lo[o] = lo;
+            a.cent16[o] = __float2half_rn(c * mul);
             if (a.cent_out) a.cent_out[o] = c;
         }
         if (tid < C) {

@@ -4,12 +4,14 @@
 // sampling sentence: blocks are drawn in proportion to the estimates and
 // re-weighted by the inverse inclusion probability).
 //
-// One CTA of 256 threads per row (query block).  The row's 48-bit
-// fixed-point weights are built once into shared memory; the water-filling
-// rounds, the Philox draws and the ordered compaction all run from there.
-// Thread t owns groups of four consecutive blocks (one Philox block yields
-// their four draws); positions in the list come from a block-wide scan of the
-// per-thread counts, so the list is ascending.  Every decision is integer
+// One CTA per row (query block).  Up to nK = 10240 the row's 48-bit
+// fixed-point weights live in registers, each thread (256 or 512 per CTA)
+// holding a contiguous run of at most 20 blocks (sample_compact_reg_kernel);
+// beyond that they are built once into shared memory (sample_compact_kernel).  The water-filling
+// rounds, the Philox draws and the ordered compaction run from there: four
+// consecutive blocks share one Philox block (one draw each), and positions in
+// the list come from a block-wide scan of the per-thread counts, so the list
+// is ascending.  Every decision is integer
 // arithmetic on the fixed-point weights: the result does not depend on the
 // launch configuration.
 #include "kernels.cuh"
@@ -222,6 +224,188 @@ __global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleAr
     }
 }
 
+// Register-resident variant for nK <= 4*G*NT: thread t owns the contiguous
+// run of blocks [t*4G, (t+1)*4G) (G Philox groups), its fixed-point weights
+// stay in registers for every water-filling round, and one block-wide scan of
+// the per-thread counts places the drawn blocks in ascending order.
+template <int NT, int G>
+__global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
+    constexpr int NW = NT / 32;
+    constexpr int PER = 4 * G;  // blocks per thread (<= 32: the masks are 32-bit)
+    // the row is staged through shared memory with coalesced loads; thread
+    // runs are SP words apart, which keeps the 16-byte reads of eight
+    // consecutive threads on distinct banks
+    constexpr int SP = (PER % 8 == 4) ? PER : PER + 4;
+    __shared__ __align__(16) float ps[NT * SP];
+    __shared__ int64_t red_w[NW];
+    __shared__ int32_t red_c[NW];
+    __shared__ int32_t wtot[NW];
+    __shared__ uint32_t sat_s[NT];  // saturation mask of each thread's run
+    const int nK = a.nK;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b0 = tid * PER;
+
+    for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
+        const float *prow = a.p + row * (int64_t)nK;
+        __syncthreads();  // the previous row is done with ps
+#pragma unroll
+        for (int u = 0; u < PER; u += 4) {
+            float v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int b = (u + q) * NT + tid;
+                v[q] = b < nK ? __ldg(prow + b) : 0.0f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int b = (u + q) * NT + tid;
+                ps[(b / PER) * SP + b % PER] = v[q];
+            }
+        }
+        __syncthreads();
+        int64_t P[PER];
+#pragma unroll
+        for (int k = 0; k < PER; k += 4) {
+            const float4 q = *reinterpret_cast<const float4 *>(ps + tid * SP + k);
+            P[k] = to_fixed48(q.x);
+            P[k + 1] = to_fixed48(q.y);
+            P[k + 2] = to_fixed48(q.z);
+            P[k + 3] = to_fixed48(q.w);
+        }
+        const int i = (int)(row % a.nQ);
+        const int64_t bh = row / a.nQ;
+        const int h = (int)(bh % a.H);
+        const int beta = (int)(bh / a.H);
+        const int nmine = max(0, min(PER, nK - b0));
+        const uint32_t valid = nmine >= 32 ? 0xffffffffu : ((1u << nmine) - 1u);
+
+        // ---- inclusion probabilities: exact water-filling (as in the shared-memory kernel)
+        uint32_t sat = 0;
+        int64_t R = a.M, T = 0;
+        if (a.M >= nK) {
+            sat = valid;
+            R = 0;
+        } else {
+            int64_t local = 0;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) local += P[k];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) local += __shfl_down_sync(0xffffffffu, local, o);
+            if (lane == 0) red_w[warp] = local;
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < NW; ++q) T += red_w[q];
+            int64_t in_s = 0;
+            for (int round = 0; round <= nK; ++round) {
+                R = a.M - in_s;
+                if (T == 0 || R <= 0) break;
+                const int64_t thr = (T + R - 1) / R;
+                int cnt = 0;
+                int64_t w = 0;
+#pragma unroll
+                for (int k = 0; k < PER; ++k) {
+                    if (!((sat >> k) & 1u) && P[k] >= thr) {
+                        sat |= 1u << k;
+                        ++cnt;
+                        w += P[k];
+                    }
+                }
+                // count and weight reduced together: one barrier pair per round
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+                    w += __shfl_down_sync(0xffffffffu, w, o);
+                }
+                __syncthreads();
+                if (lane == 0) {
+                    red_c[warp] = cnt;
+                    red_w[warp] = w;
+                }
+                __syncthreads();
+                int added = 0;
+                int64_t added_w = 0;
+#pragma unroll
+                for (int q = 0; q < NW; ++q) {
+                    added += red_c[q];
+                    added_w += red_w[q];
+                }
+                if (added == 0) break;
+                in_s += added;
+                T -= added_w;
+            }
+        }
+        sat &= valid;
+
+        // ---- draws: group g = tid*G + u gives blocks 4g..4g+3 ----------------
+        uint32_t take = 0;
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            const int g = tid * G + u;
+            if (4 * g >= nK) break;
+            const uint4 r4 =
+                philox4x32_10(make_uint4((uint32_t)g, (uint32_t)i, (uint32_t)h, (uint32_t)beta), a.key0, a.key1);
+            const uint32_t U[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int bit = 4 * u + k;
+                if (!((valid >> bit) & 1u)) continue;
+                if ((sat >> bit) & 1u) {
+                    take |= 1u << bit;
+                } else {
+                    const uint64_t rp = (uint64_t)(R * P[bit]);
+                    if (rp != 0 && draw_below(U[k], (uint64_t)T, rp)) take |= 1u << bit;
+                }
+            }
+        }
+        // ---- ordered compaction: exclusive scan of the per-thread counts -------
+        const int cnt = __popc(take);
+        int x = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        __syncthreads();  // wtot reuse guard
+        if (lane == 31) wtot[warp] = x;
+        __syncthreads();
+        int pos = x - cnt, total = 0;
+#pragma unroll
+        for (int q = 0; q < NW; ++q) {
+            const int c = wtot[q];
+            pos += q < warp ? c : 0;
+            total += c;
+        }
+        int32_t *idx_row = a.idx + row * (int64_t)a.capacity;
+        float *logw_row = a.logw + row * (int64_t)a.capacity;
+        // static indices keep P in registers
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            if (!((take >> k) & 1u)) continue;
+            if (pos < a.capacity) idx_row[pos] = b0 + k;
+            ++pos;
+        }
+        sat_s[tid] = sat;
+        const int n = min(total, a.capacity);
+        if (tid == 0) {
+            if (total > a.capacity) raise_flag(a.status, ABATT_DEVFLAG_CAPACITY);
+            a.counts[row] = n;
+        }
+        __syncthreads();  // the list and the saturation masks are complete
+        // log-weights in a second, convergent pass: list entry j on thread
+        // j mod NT, its weight re-derived from the staged row
+        for (int j = tid; j < n; j += NT) {
+            const int b = idx_row[j];
+            const int owner = b / PER, k = b - owner * PER;
+            float lw = 0.0f;
+            if (!((sat_s[owner] >> k) & 1u)) {
+                const int64_t rp = R * to_fixed48(ps[owner * SP + k]);
+                lw = (float)(-log((double)rp / (double)T));
+            }
+            logw_row[j] = lw;
+        }
+    }
+}
+
 }  // namespace
 
 size_t sample_smem_bytes(int nK) {
@@ -230,11 +414,35 @@ size_t sample_smem_bytes(int nK) {
 }
 
 cudaError_t launch_sample(const SampleArgs &a, int num_sms, cudaStream_t stream) {
-    const size_t smem = sample_smem_bytes(a.nK);
     int64_t grid = a.rows;
+    if (grid < 1) return cudaSuccess;
+    // register-resident kernel: at most five Philox groups (20 blocks) per
+    // thread, with 256 threads up to nK = 5120 and 512 up to 10240
+    const int G256 = (a.nK + 1023) / 1024, G512 = (a.nK + 2047) / 2048;
+    if (G256 <= 5 || G512 <= 5) {
+        const int64_t cap = (int64_t)num_sms * (G256 <= 5 ? 8 : 4);
+        if (grid > cap) grid = cap;
+        const unsigned gr = (unsigned)grid;
+        if (G256 <= 5) {
+            switch (G256) {
+                case 1: sample_compact_reg_kernel<256, 1><<<gr, 256, 0, stream>>>(a); break;
+                case 2: sample_compact_reg_kernel<256, 2><<<gr, 256, 0, stream>>>(a); break;
+                case 3: sample_compact_reg_kernel<256, 3><<<gr, 256, 0, stream>>>(a); break;
+                case 4: sample_compact_reg_kernel<256, 4><<<gr, 256, 0, stream>>>(a); break;
+                default: sample_compact_reg_kernel<256, 5><<<gr, 256, 0, stream>>>(a); break;
+            }
+        } else if (G512 <= 3) {
+            sample_compact_reg_kernel<512, 3><<<gr, 512, 0, stream>>>(a);
+        } else if (G512 == 4) {
+            sample_compact_reg_kernel<512, 4><<<gr, 512, 0, stream>>>(a);
+        } else {
+            sample_compact_reg_kernel<512, 5><<<gr, 512, 0, stream>>>(a);
+        }
+        return cudaGetLastError();
+    }
+    const size_t smem = sample_smem_bytes(a.nK);
     const int64_t cap = (int64_t)num_sms * 64;
     if (grid > cap) grid = cap;
-    if (grid < 1) return cudaSuccess;
     cudaError_t e;
     if (a.nK <= kCacheMaxBlocks) {
         e = cudaFuncSetAttribute(sample_compact_kernel<true>,

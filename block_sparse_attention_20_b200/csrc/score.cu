@@ -3,15 +3,20 @@
 // Block Attention", abstract, selector sentence: the clustered queries
 // estimate block importance).
 //
-// score_mass_kernel: one CTA per (head, 128 centroid rows).  The centroid
-// tile (bf16 hi + lo split of the pre-scaled fp32 centroids) stays in shared
-// memory; 128-key tiles of K stream through a 4-stage TMA ring; one thread
-// issues tcgen05 MMAs into a double-buffered 128x128 fp32 accumulator in
-// tensor memory; two epilogue warpgroups (one per accumulator buffer, thread
-// = centroid row) turn each tile into base-2 exponentials relative to the
-// row's running maximum and sum them per key block.  The partial block sums
-// of a tile are written with the reference maximum they were taken against,
-// so no second pass over the keys is needed.
+// keys_f16_kernel: the keys once to fp16, the scoring GEMM's B operand.
+//
+// score_mass_kernel: one CTA per (head, 128 centroid rows, key-range chunk).
+// The centroid tile (fp16 of the pre-scaled fp32 centroids: 11 significant
+// bits, against 8 for bf16) stays in shared memory; 128-key fp16 tiles of K
+// stream through a 4-stage TMA ring; one warp issues tcgen05 MMAs
+// (kind::f16, fp32 accumulation) into a double-buffered 128x128 accumulator
+// in tensor memory; two epilogue warpgroups (one per accumulator buffer,
+// thread = centroid row) turn each tile into base-2 exponentials relative to
+// the row's running maximum and sum them per key block, two values per
+// packed fp32 instruction, with a fixed share of the exponentials on the FMA
+// pipe (polynomial) and the rest on the special-function unit.  The partial
+// block sums of a tile are written with the reference maximum they were
+// taken against, so no second pass over the keys is needed.
 //
 // combine_kernel: one CTA per query block:
 //   p_b = sum_j (n_j/n) * r_{j,b} * 2^(mref_{j,T(b)} - m_j) / Z_j
@@ -25,6 +30,34 @@ namespace {
 constexpr int kScoreStages = 4;
 constexpr int kScoreThreads = 320;  // warps 0-7 epilogue (2 warpgroups), 8 TMA, 9 MMA
 #define kNegInf (-__int_as_float(0x7f800000))
+// exponent pairs of every sixteen that the epilogue evaluates with the
+// FMA-pipe polynomial (the others use ex2)
+#ifndef ABATT_SCORE_POLY_OF_16
+#define ABATT_SCORE_POLY_OF_16 7
+#endif
+constexpr int kScorePolyOf16 = ABATT_SCORE_POLY_OF_16;
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_sat(uint32_t w) {
+    const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.0f), 65504.0f);
+    const float hi = fminf(fmaxf(__uint_as_float(w & 0xffff0000u), -65504.0f), 65504.0f);
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__global__ void __launch_bounds__(256) keys_f16_kernel(const uint4 *__restrict__ src,
+                                                       uint4 *__restrict__ dst, int64_t n8) {
+    const int64_t stride = (int64_t)gridDim.x * 256;
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += 2 * stride) {
+        const bool two = i + stride < n8;
+        const uint4 u0 = __ldg(src + i);
+        const uint4 u1 = two ? __ldg(src + i + stride) : make_uint4(0, 0, 0, 0);
+        dst[i] = make_uint4(bf16x2_to_f16x2_sat(u0.x), bf16x2_to_f16x2_sat(u0.y),
+                            bf16x2_to_f16x2_sat(u0.z), bf16x2_to_f16x2_sat(u0.w));
+        if (two)
+            dst[i + stride] = make_uint4(bf16x2_to_f16x2_sat(u1.x), bf16x2_to_f16x2_sat(u1.y),
+                                         bf16x2_to_f16x2_sat(u1.z), bf16x2_to_f16x2_sat(u1.w));
+    }
+}
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -53,9 +86,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *sA_hi = smem;
-    uint8_t *sA_lo = smem + TILE;
-    uint8_t *sK = smem + 2 * TILE;
+    uint8_t *sA = smem;
+    uint8_t *sK = smem + TILE;
 
     __shared__ __align__(8) uint64_t bar_a;
     __shared__ __align__(8) uint64_t bar_kfull[ST], bar_kempty[ST];
@@ -102,13 +134,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
-            tma_prefetch_desc(&maps.a_hi);
+            tma_prefetch_desc(&maps.a);
             tma_prefetch_desc(&maps.k);
-            mbar_arrive_expect_tx(&bar_a, (a.use_lo ? 2u : 1u) * TILE);
-            for (int c = 0; c < CH; ++c) {
-                tma_load_3d(sA_hi + c * 16384, &maps.a_hi, &bar_a, c * 64, mt * 128, hd);
-                if (a.use_lo) tma_load_3d(sA_lo + c * 16384, &maps.a_lo, &bar_a, c * 64, mt * 128, hd);
-            }
+            mbar_arrive_expect_tx(&bar_a, TILE);
+            for (int c = 0; c < CH; ++c) tma_load_3d(sA + c * 16384, &maps.a, &bar_a, c * 64, mt * 128, hd);
             for (int i = 0; i < ntl; ++i) {
                 const int s = i % ST;
                 if (i >= ST && !mbar_wait(&bar_kempty[s], ((i / ST) - 1) & 1, wc, 0x101)) break;
@@ -127,10 +156,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         };
         if (wait_all(&bar_a, 0, 0x102)) {
             tc_fence_after();
-            constexpr uint32_t idesc = idesc_bf16(128, 128);
-            const uint32_t a_hi = smem_u32(sA_hi), a_lo = smem_u32(sA_lo);
-            const uint64_t dhi = sdesc_sw128(a_hi, 16, 1024), dlo = sdesc_sw128(a_lo, 16, 1024);
-            const bool use_lo = a.use_lo != 0;
+            constexpr uint32_t idesc = idesc_f16(128, 128);
+            const uint64_t da = sdesc_sw128(smem_u32(sA), 16, 1024);
             for (int i = 0; i < ntl; ++i) {
                 const int s = i % ST, buf = i & 1, use = i >> 1;
                 if (!wait_all(&bar_kfull[s], (i / ST) & 1, 0x103)) break;
@@ -141,8 +168,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                    umma_bf16_ss_w(d_tmem, dhi + off, kd + off, idesc, kk > 0);
-                    if (use_lo) umma_bf16_ss_w(d_tmem, dlo + off, kd + off, idesc, 1);
+                    umma_ss_w(d_tmem, da + off, kd + off, idesc, kk > 0);
                 }
                 umma_commit_w(&bar_kempty[s]);
                 umma_commit_w(&bar_sfull[buf]);
@@ -182,24 +208,54 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     for (int c = 0; c < 32; ++c)
                         if (q * 32 + c >= nvalid) v[q][c] = __float_as_uint(kNegInf);
             }
-            float tm = kNegInf;
+            // four independent max chains (one per 32-column load), then merged
+            float tq[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 4; ++q) {
+                tq[q] = kNegInf;
 #pragma unroll
                 for (int c = 0; c < 32; c += 2)
-                    tm = fmax3f(tm, __uint_as_float(v[q][c]), __uint_as_float(v[q][c + 1]));
+                    tq[q] = fmax3f(tq[q], __uint_as_float(v[q][c]), __uint_as_float(v[q][c + 1]));
+            }
+            const float tm = fmaxf(fmax3f(tq[0], tq[1], tq[2]), tq[3]);
             const float m_new = fmaxf(m_run, tm);
             const float alpha = (m_run == kNegInf) ? 0.0f : ex2_approx(m_run - m_new);
             Z *= alpha;
             m_run = m_new;
-            float bs[BPT];
+            // 2^(x - m) two columns at a time; NA interleaved partial sums per
+            // block keep the add chains short when blocks are wide
+            constexpr int NA = BPT >= 8 ? 1 : 8 / BPT;
+            const float2 nm = make_float2(-m_run, -m_run);
+            float2 acc[BPT][NA];
 #pragma unroll
-            for (int k = 0; k < BPT; ++k) bs[k] = 0.0f;
+            for (int k = 0; k < BPT; ++k)
+#pragma unroll
+                for (int u = 0; u < NA; ++u) acc[k][u] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    bs[(q * 32 + c) / BK] += ex2_approx(__uint_as_float(v[q][c]) - m_run);
+                for (int c = 0; c < 32; c += 2) {
+                    const int col = q * 32 + c;
+                    const float2 x =
+                        __fadd2_rn(make_float2(__uint_as_float(v[q][c]), __uint_as_float(v[q][c + 1])), nm);
+                    float2 e;
+                    if (((col >> 1) & 15) < kScorePolyOf16) {
+                        e = exp2_poly2<4>(x);
+                    } else {
+                        e.x = ex2_approx(x.x);
+                        e.y = ex2_approx(x.y);
+                    }
+                    float2 &s2 = acc[col / BK][(col >> 1) % NA];
+                    s2 = __fadd2_rn(s2, e);
+                }
+            float bs[BPT];
+#pragma unroll
+            for (int k = 0; k < BPT; ++k) {
+                float2 t2 = acc[k][0];
+#pragma unroll
+                for (int u = 1; u < NA; ++u) t2 = __fadd2_rn(t2, acc[k][u]);
+                bs[k] = t2.x + t2.y;
+            }
 #pragma unroll
             for (int k = 0; k < BPT; ++k) Z += bs[k];
             if (valid) {
@@ -320,7 +376,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 
 template <int D, int BK>
 cudaError_t launch_score_t(const ScoreArgs &a, const ScoreMaps &maps, cudaStream_t stream) {
-    const size_t smem = (2 + kScoreStages) * (size_t)(128 * D * 2) + 1024;
+    const size_t smem = (1 + kScoreStages) * (size_t)(128 * D * 2) + 1024;
     cudaError_t e = cudaFuncSetAttribute(score_mass_kernel<D, BK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -345,6 +401,17 @@ cudaError_t launch_score_d(const ScoreArgs &a, const ScoreMaps &maps, cudaStream
 cudaError_t launch_score(const ScoreArgs &a, const ScoreMaps &maps, int, cudaStream_t stream) {
     if (a.heads < 1 || a.MC < 1 || a.nT < 1) return cudaSuccess;
     return a.D == 128 ? launch_score_d<128>(a, maps, stream) : launch_score_d<64>(a, maps, stream);
+}
+
+cudaError_t launch_keys_f16(const __nv_bfloat16 *K, __half *K16, int64_t n8, int num_sms,
+                            cudaStream_t stream) {
+    if (n8 < 1) return cudaSuccess;
+    int64_t grid = (n8 + 511) / 512;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (grid > cap) grid = cap;
+    keys_f16_kernel<<<(unsigned)grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(K),
+                                                        reinterpret_cast<uint4 *>(K16), n8);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const CombineArgs &a, int num_sms, cudaStream_t stream) {

@@ -72,7 +72,9 @@ def _rows_of(shape, Bq=128):
                                            (7425, 16, 1100, 0.2), (63, 16, 2500, 1.0),
                                            (8192, 16, 500, 0.1), (1, 128, 1000, 1.0),
                                            (3, 64, 9000, 0.5), (64, 32, 10000, 0.3),
-                                           (100, 16, 0, 0.3)])
+                                           (100, 16, 0, 0.3), (1500, 16, 1200, 0.2), (10300, 16, 700, 0.1),
+                                           (2900, 16, 900, 0.1), (5500, 16, 700, 0.1),
+                                           (9001, 16, 800, 0.1)])
 def test_sample_bit_exact(nK, Bk, bp, conc):
     N = nK * Bk - (Bk // 2 if nK > 1 else 0)
     shape = (1, 2, N, 64)
