@@ -19,12 +19,14 @@
 //
 //   tensor core, per tile t:   S0(t)  PV1(t-1)  S1(t)  PV0(t)
 //
-// Warp roles (576 threads):
+// Warp roles (640 threads, five warpgroups; warpgroup 0 hands registers to
+// the softmax warpgroups with setmaxnreg):
 //   warp 0      TMA producer: Q of both rows, then K(t), V(t) into a ring;
 //   warp 1      tensor-memory owner and tcgen05 MMA issuer:
 //               S_s = Q_s K^T (fp32, 128 TMEM columns per row),
 //               O_s += P_s V  (P_s read back from the columns S_s used);
-//   warps 2-17  softmax, eight warps per row s of the pair; a warp owns 16
+//   warps 2-3   idle;
+//   warps 4-19  softmax, eight warps per row s of the pair; a warp owns 16
 //               query rows of its tensor-memory lane quarter and its two
 //               half-warps split each row's 128 columns (two threads per
 //               query): raw per-block maxima of the thread's 64 columns, the
@@ -41,7 +43,9 @@ namespace abatt {
 
 namespace {
 
-constexpr int kAttnThreads = 576;
+constexpr int kAttnThreads = 640;   // warpgroup 0: TMA, MMA (+2 idle warps); 1-4: softmax
+constexpr int kRegsControl = 56;     // registers per thread of warpgroup 0 after setmaxnreg
+constexpr int kRegsSoftmax = 104;    // ... and of the four softmax warpgroups
 #define kNegInf (-__int_as_float(0x7f800000))
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -49,7 +53,7 @@ constexpr float kRescaleThreshold = 8.0f;
 // exponent pairs of every eight that the softmax evaluates with the FMA-pipe
 // polynomial (the others use ex2); balances the two pipes
 #ifndef ABATT_ATTN_POLY_OF_8
-#define ABATT_ATTN_POLY_OF_8 3
+#define ABATT_ATTN_POLY_OF_8 0
 #endif
 constexpr int kAttnPolyOf8 = ABATT_ATTN_POLY_OF_8;
 
@@ -278,6 +282,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t ring_issued = 0;  // producer: ring loads issued (for the drain)
 
     if (warp == 0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
         // ================================ TMA producer ================================
         // The whole warp: lane 0 owns the barriers; lane k < 128/Bk gathers
         // block k of each tile, its index prefetched one tile ahead.
@@ -358,6 +363,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
         }
     } else if (warp == 1) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
         // ================================ MMA issuer ==================================
         // The whole warp runs the schedule, so its control flow and the
         // descriptors stay warp-uniform; one elected lane issues each tcgen05
@@ -451,13 +457,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             rp = base + 2u * (uint32_t)P.groups;
         }
-    } else if (warp >= 2) {
+    } else if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));  // idle
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ================================ softmax =====================================
         // Eight warps per row of the pair.  A warp owns 16 query rows (TMEM
         // lanes) of its lane quarter; the two half-warps split each row's
         // columns, so a row's maximum and sum need one shuffle, not a barrier.
         constexpr int HB = BPT >= 2 ? BPT / 2 : 1;  // blocks (or block parts) per column half
-        const int sw = warp - 2;
+        const int sw = warp - 4;
         const int s = sw >> 3;              // row of the pair
         const int sub = (sw >> 2) & 1;      // 16-lane half of the lane quarter
         const int wq = warp & 3;            // tensor-memory lane quarter
@@ -481,6 +490,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
             const float *lw = a.ulw + (pr * 2 + s) * (int64_t)a.cap_u;
             float m_run = kNegInf, l = 0.0f;
+            // raw log-weights and block ids of this half's blocks for the next
+            // tile, loaded one tile ahead and first read at that tile (their
+            // latency hides behind the current tile)
+            float nw[HB];
+            int nbk[HB];
+            auto load_meta = [&](int t) {
+#pragma unroll
+                for (int k = 0; k < HB; ++k) {
+                    const int e = t * BPT + (BPT >= 2 ? hh * HB + k : 0);
+                    nw[k] = -1.0f;  // empty slot: not drawn
+                    nbk[k] = 0;
+                    if (e < U) {
+                        const int j = P.pos(s, e);
+                        nw[k] = __ldg(lw + j);
+                        nbk[k] = __ldg(ub + j);
+                    }
+                }
+            };
+            if (n > 0) load_meta(0);
             for (int t = 0; t < n; ++t) {
                 // this half's blocks: base-2 log-weight (-inf where this row did
                 // not draw the block or the slot is empty); the block that can
@@ -489,19 +517,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 int tail_k = -1, tail_keep = BK;
 #pragma unroll
                 for (int k = 0; k < HB; ++k) {
-                    const int e = t * BPT + (BPT >= 2 ? hh * HB + k : 0);
-                    bias[k] = kNegInf;
-                    if (e < U) {
-                        const int j = P.pos(s, e);
-                        const float w = __ldg(lw + j);
-                        if (w >= 0.0f) bias[k] = w * kLog2e;
-                        const int b = __ldg(ub + j);
-                        if (b == a.nK - 1 && a.N - b * BK < BK) {
-                            tail_k = k;
-                            tail_keep = a.N - b * BK;
-                        }
+                    const float w = nw[k];
+                    const int b = nbk[k];
+                    bias[k] = w >= 0.0f ? w * kLog2e : kNegInf;
+                    if (w >= 0.0f && b == a.nK - 1 && a.N - b * BK < BK) {
+                        tail_k = k;
+                        tail_keep = a.N - b * BK;
                     }
                 }
+                if (t + 1 < n) load_meta(t + 1);
                 const bool masked = tail_k >= 0;
                 if (!mbar_wait(&bar_sf[s], s_uses & 1, wc, 0x208)) { ok = false; break; }
                 ++s_uses;
@@ -669,6 +693,14 @@ cudaError_t launch_attn_t(const AttnArgs &a, const AttnMaps &maps, int num_sms, 
     cudaError_t e = cudaFuncSetAttribute(gather_attn_kernel<D, BK, KF>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    // setmaxnreg moves registers between warpgroups within the launch's
+    // allocation: the compiled count must cover the split, else the
+    // increase would never be granted
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, gather_attn_kernel<D, BK, KF>);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)fa.numRegs * kAttnThreads < 128 * kRegsControl + (kAttnThreads - 128) * kRegsSoftmax)
+        return cudaErrorInvalidConfiguration;
     const int grid = (int)(a.pairs < num_sms ? a.pairs : num_sms);
     gather_attn_kernel<D, BK, KF><<<grid, kAttnThreads, smem, stream>>>(maps, a);
     return cudaGetLastError();
