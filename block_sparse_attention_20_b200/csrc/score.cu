@@ -33,7 +33,7 @@ constexpr int kScoreThreads = 320;  // warps 0-7 epilogue (2 warpgroups), 8 TMA,
 // exponent pairs of every sixteen that the epilogue evaluates with the
 // FMA-pipe polynomial (the others use ex2)
 #ifndef ABATT_SCORE_POLY_OF_16
-#define ABATT_SCORE_POLY_OF_16 7
+#define ABATT_SCORE_POLY_OF_16 4
 #endif
 constexpr int kScorePolyOf16 = ABATT_SCORE_POLY_OF_16;
 
