@@ -48,6 +48,27 @@ def parse():
     return ap.parse_args()
 
 
+def attention_traffic(rows: int):
+    """DRAM bytes of one gather_attn_kernel launch, from the committed ncu
+    summary (bytes per query block, scaled by the launch's query blocks; DRAM
+    traffic of the kernel is its compulsory Q/K/V/O bytes, which grow with the
+    query blocks).  None when the kernel source differs from the one the
+    counters were taken on."""
+    import hashlib
+    import re
+    csrc = os.path.join(ROOT, "block_sparse_attention_20_b200", "csrc")
+    try:
+        src = b"".join(open(os.path.join(csrc, f), "rb").read()
+                       for f in ("attention.cu", "common.cuh", "kernels.cuh"))
+        txt = open(os.path.join(ROOT, "profiles", "gather_attn_kernel_wan1.3b.md")).read()
+    except OSError:
+        return None
+    m = re.search(r"source sha256 ([0-9a-f]{16}); DRAM bytes per query block: ([0-9]+)", txt)
+    if not m or m.group(1) != hashlib.sha256(src).hexdigest()[:16]:
+        return None
+    return int(m.group(2)) * rows
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -296,7 +317,7 @@ def main():
         "executed_tflops_attention": exec_flop / (att_mean * 1e-3) / 1e12,
         "algorithmic_tflops_attention": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": attention_traffic(rows),
                      "kernel": "gather_attn_kernel", "flops": "algorithmic (valid query rows x drawn keys)",
                      "peak_source": f"{src} bf16 sustained"},
         "device_status": status,
