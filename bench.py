@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-keep-all", action="store_true", help="skip the keep-all attention timing")
+    ap.add_argument("--e2e-heads", type=int, default=2, help="heads per chunk of the host pipeline")
     return ap.parse_args()
 
 
@@ -366,25 +367,20 @@ def keep_all(abatt, cfg, Q, K, V, w, O, ws, stream):
 
 
 def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):
-    """Same metric through the public call with host buffers: pinned H2D of
-    Q, K, V, abatt_forward, D2H of O, every step."""
+    """Same metric through the public host-to-host call: every step copies
+    Q, K, V from pinned host memory to the device and O back, through
+    abatt.HostPipeline (abatt_forward over chunks of heads, the copies of one
+    chunk overlapped with the compute of the previous one)."""
     import torch
     import torch.distributed as dist
 
     hq, hk, hv = (t.pin_memory() for t in (Qc, Kc, Vc))
     ho = torch.empty_like(Qc).pin_memory()
-    Q, K, V = (torch.empty_like(t, device=dev) for t in (Qc, Kc, Vc))
-    O = torch.empty_like(Q)
-    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, w.shape, cfg), dtype=torch.uint8,
-                     device=dev)
+    pipe = abatt.HostPipeline(w.shape, cfg, heads_per_chunk=args.e2e_heads, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        Q.copy_(hq, non_blocking=True)
-        K.copy_(hk, non_blocking=True)
-        V.copy_(hv, non_blocking=True)
-        abatt.forward(Q, K, V, cfg, out=O, workspace=ws, stream=stream)
-        ho.copy_(O, non_blocking=True)
+        pipe(hq, hk, hv, ho)
 
     steps = max(3, args.steps // 4)
     for _ in range(3):
@@ -408,7 +404,7 @@ def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):
     nbytes = Qc.numel() * 2
     return {"value": dense * world / (ms * 1e-3) / 1e12, "unit": "TFLOPS (dense-equivalent)",
             "ms_per_step": ms, "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
-            "steps": steps}
+            "steps": steps, "heads_per_chunk": pipe.hc, "device_status": pipe.status()}
 
 
 if __name__ == "__main__":

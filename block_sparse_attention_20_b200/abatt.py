@@ -43,7 +43,8 @@ class _Shape(ctypes.Structure):
 class _Config(ctypes.Structure):
     _fields_ = [("q_block", ctypes.c_int), ("kv_block", ctypes.c_int), ("clusters", ctypes.c_int),
                 ("kmeans_iters", ctypes.c_int), ("budget_bp", ctypes.c_int),
-                ("scale", ctypes.c_float), ("seed", ctypes.c_uint64)]
+                ("scale", ctypes.c_float), ("seed", ctypes.c_uint64),
+                ("batch_offset", ctypes.c_int), ("head_offset", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -57,11 +58,13 @@ class Config:
     budget_bp: int = 1000
     scale: float | None = None  # default 1/sqrt(d)
     seed: int = 0
+    batch_offset: int = 0  # global index of the call's first batch element
+    head_offset: int = 0   # global index of the call's first head
 
     def _c(self, d: int) -> _Config:
         s = self.scale if self.scale is not None else 1.0 / math.sqrt(d)
         return _Config(self.q_block, self.kv_block, self.clusters, self.kmeans_iters,
-                       self.budget_bp, s, self.seed & (2**64 - 1))
+                       self.budget_bp, s, self.seed & (2**64 - 1), self.batch_offset, self.head_offset)
 
 
 _lock = threading.Lock()
@@ -257,6 +260,74 @@ def forward(q, k, v, cfg: Config, *, out=None, want_lse=False, workspace=None, s
                                ctypes.byref(cfg._c(sh.d)), _ptr(out), _ptr(lse), _ptr(ws),
                                ws.numel(), _stream(stream)), "abatt_forward")
     return (out, lse) if want_lse else out
+
+
+class HostPipeline:
+    """The whole path on pinned host tensors, with the copies overlapped.
+
+    Heads are independent and the sampler draws with global head indices
+    (``Config.head_offset``), so the problem is split into chunks of
+    ``heads_per_chunk`` heads of one batch element; while chunk j runs
+    ``abatt_forward`` on the compute stream, chunk j+1's Q, K, V travel
+    host -> device on a copy stream and chunk j-1's O travels back on a third.
+    The result equals one ``forward`` over the whole problem.  Device buffers
+    (two chunk sets) and one FORWARD workspace per chunk are allocated once,
+    here; every chunk's status word stays readable (:meth:`status`).
+    """
+
+    def __init__(self, shape, cfg: Config, *, heads_per_chunk: int = 5, device=None):
+        import torch
+        self.B, self.H, self.N, self.d = shape
+        self.cfg = cfg
+        self.hc = max(1, min(heads_per_chunk, self.H))
+        self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.chunks = [(b, h0, min(h0 + self.hc, self.H)) for b in range(self.B)
+                       for h0 in range(0, self.H, self.hc)]
+        cshape = (1, self.hc, self.N, self.d)
+        self.buf = [[torch.empty(cshape, dtype=torch.bfloat16, device=self.dev) for _ in range(4)]
+                    for _ in range(2)]  # (Q, K, V, O) x 2
+        self.ws = [torch.empty(workspace_size(CALL_FORWARD, (1, h1 - h0, self.N, self.d), cfg),
+                               dtype=torch.uint8, device=self.dev) for _, h0, h1 in self.chunks]
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(self.dev) for _ in range(3))
+
+    def __call__(self, q, k, v, out):
+        """q, k, v, out: pinned host bf16 [B, H, N, d].  Enqueues everything;
+        the current stream waits for the last copy of O."""
+        import torch
+        n = len(self.chunks)
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_comp = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        self.s_in.wait_stream(torch.cuda.current_stream(self.dev))
+        for j, (b, h0, h1) in enumerate(self.chunks):
+            Qd, Kd, Vd, Od = (t[:, :h1 - h0] for t in self.buf[j % 2])
+            with torch.cuda.stream(self.s_in):
+                if j >= 2:
+                    self.s_in.wait_event(ev_out[j - 2])  # buffer set free again
+                Qd.copy_(q[b:b + 1, h0:h1], non_blocking=True)
+                Kd.copy_(k[b:b + 1, h0:h1], non_blocking=True)
+                Vd.copy_(v[b:b + 1, h0:h1], non_blocking=True)
+                ev_in[j].record(self.s_in)
+            self.s_comp.wait_event(ev_in[j])
+            c = Config(**{**self.cfg.__dict__, "batch_offset": self.cfg.batch_offset + b,
+                          "head_offset": self.cfg.head_offset + h0})
+            forward(Qd, Kd, Vd, c, out=Od, workspace=self.ws[j], stream=self.s_comp)
+            ev_comp[j].record(self.s_comp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ev_comp[j])
+                out[b:b + 1, h0:h1].copy_(Od, non_blocking=True)
+                ev_out[j].record(self.s_out)
+        torch.cuda.current_stream(self.dev).wait_event(ev_out[n - 1])
+        for e in ev_out[:-1]:
+            torch.cuda.current_stream(self.dev).wait_event(e)
+        return out
+
+    def status(self) -> int:
+        """OR of every chunk's device status word (synchronises)."""
+        f = 0
+        for w in self.ws:
+            f |= read_status(w)
+        return f
 
 
 def intermediates(workspace, shape, cfg: Config):

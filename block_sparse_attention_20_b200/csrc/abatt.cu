@@ -50,6 +50,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (!s || !c) return ABATT_ERR_INVALID_ARG;
     if (s->B <= 0 || s->H <= 0 || s->N <= 0 || s->d <= 0) return ABATT_ERR_INVALID_ARG;
     if (c->budget_bp < 0 || !(c->scale > 0.0f) || !isfinite(c->scale)) return ABATT_ERR_INVALID_ARG;
+    if (c->batch_offset < 0 || c->head_offset < 0) return ABATT_ERR_INVALID_ARG;
     if (s->d != 64 && s->d != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->q_block != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->kv_block != 16 && c->kv_block != 32 && c->kv_block != 64 && c->kv_block != 128)
@@ -241,6 +242,8 @@ abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, 
     SampleArgs a;
     a.p = p; a.rows = g.rows; a.nK = g.nK; a.nK_pad = (g.nK + 3) & ~3; a.nQ = g.nQ; a.H = g.H;
     a.M = g.M;
+    a.b_off = (uint32_t)cfg->batch_offset;
+    a.h_off = (uint32_t)cfg->head_offset;
     a.key0 = (uint32_t)(cfg->seed & 0xffffffffu);
     a.key1 = (uint32_t)(cfg->seed >> 32);
     a.capacity = capacity; a.counts = counts; a.idx = idx; a.logw = logw;

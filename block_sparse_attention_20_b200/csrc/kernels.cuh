@@ -66,6 +66,7 @@ struct SampleArgs {
     int64_t rows;
     int nK, nK_pad, nQ, H;
     int64_t M;
+    uint32_t b_off, h_off;  // global index of the first batch element / head (Philox counter)
     uint32_t key0, key1;
     int capacity;
     int32_t *counts, *idx;

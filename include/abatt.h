@@ -77,6 +77,12 @@ typedef struct abatt_config {
                            keeps every block with weight 1 */
     float scale;        /* softmax scale s (1/sqrt(d) for plain attention) */
     uint64_t seed;      /* Philox key for the draws */
+    int batch_offset;   /* global index of this call's first batch element (0 for a whole tensor) */
+    int head_offset;    /* global index of this call's first head (0 for a whole tensor) */
+    /* The sampler's Philox counter uses the global indices (beta + batch_offset,
+       h + head_offset), so a call over a slice of the batches or heads of a
+       larger problem draws exactly the blocks that one call over the whole
+       problem draws for that slice.  Both must be >= 0 (ABATT_ERR_INVALID_ARG). */
 } abatt_config;
 
 /* Which call a workspace is for. */

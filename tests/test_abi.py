@@ -71,6 +71,8 @@ def test_workspace_sizes():
     ((1, 1, 100, 64), {"budget_bp": -1}, 1),
     ((1, 1, 100, 64), {"scale": 0.0}, 1),
     ((1, 1, 100, 64), {"scale": float("nan")}, 1),
+    ((1, 1, 100, 64), {"head_offset": -1}, 1),
+    ((1, 1, 100, 64), {"batch_offset": -3}, 1),
 ])
 def test_validation(shape, kw, code):
     with pytest.raises(abatt.AbattError) as e:
@@ -116,3 +118,11 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(abatt, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         abatt.lib()
+
+
+def test_config_struct_carries_the_slice_offsets():
+    # abatt_config ends with batch_offset, head_offset after the 64-bit seed
+    c = abatt.Config(seed=5, batch_offset=2, head_offset=7)._c(64)
+    assert ctypes.sizeof(c) == 40
+    assert (c.seed, c.batch_offset, c.head_offset) == (5, 2, 7)
+    assert abatt._Config.head_offset.offset == 36 and abatt._Config.batch_offset.offset == 32

@@ -109,6 +109,25 @@ def test_sample_capacity_overflow_flags_and_truncates():
         assert np.array_equal(i[r], oi[r, :cap])
 
 
+def test_sample_head_slice_draws_like_the_whole_call():
+    # a call over heads [1, 3) of a 3-head problem, with head_offset = 1, draws
+    # bit for bit what the 3-head call draws for those heads
+    nK, Bk = 700, 16
+    shape = (1, 3, nK * Bk, 64)
+    nQ = -(-shape[2] // 128)
+    p = torch.from_numpy(synth.random_probs(3 * nQ, nK, 21, 0.2)).cuda()
+    cfg = abatt.Config(kv_block=Bk, budget_bp=900, seed=77)
+    c, i, lw, _ = abatt.sample(p, shape, cfg)
+    cs, is_, lws, _ = abatt.sample(p[nQ:].contiguous(), (1, 2, shape[2], 64),
+                                   abatt.Config(kv_block=Bk, budget_bp=900, seed=77, head_offset=1))
+    assert torch.equal(cs, c[nQ:])
+    c = c.cpu().numpy()
+    for r in range(2 * nQ):
+        L = c[nQ + r]
+        assert torch.equal(is_[r, :L], i[nQ + r, :L])
+        assert torch.equal(lws[r, :L].view(torch.int32), lw[nQ + r, :L].view(torch.int32))
+
+
 def test_sample_repeatable_on_other_stream():
     nK, Bk = 4725, 16
     shape = (1, 3, nK * Bk, 128)
@@ -344,3 +363,37 @@ def test_forward_wan14b_full_size_sampled_rows():
     rows = [h * nQ + i for h, i in [(0, 0), (0, nQ - 1), (7, 100), (13, 295), (21, 1), (27, 400),
                                     (33, 590), (39, 0), (39, 333), (39, nQ - 1)]]
     _forward_check(w, rows)
+
+
+def test_host_pipeline_matches_one_forward():
+    # pinned host Q/K/V -> O through head chunks with overlapped copies equals
+    # one forward over all heads (the draws use global head indices)
+    w = synth.WAN_1_3B.with_(H=5, N=3000, grid=(3, 20, 50))
+    Q, K, V = synth.generate(w)
+    shape = (1, 5, w.N, w.d)
+    cfg = cfg_of(w)
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, shape, cfg), dtype=torch.uint8,
+                     device="cuda")
+    O1 = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg, workspace=ws)
+    _, c1, i1, _ = (t.cpu().numpy() for t in abatt.intermediates(ws, shape, cfg))
+    pipe = abatt.HostPipeline(shape, cfg, heads_per_chunk=2)
+    hq, hk, hv = (t.pin_memory() for t in (Q, K, V))
+    ho = torch.empty_like(Q).pin_memory()
+    pipe(hq, hk, hv, ho)
+    torch.cuda.synchronize()
+    assert pipe.status() == 0 and abatt.read_status(ws) == 0
+    # the same blocks drawn, chunk by chunk
+    nQ = w.nQ
+    diff = tot = 0
+    for j, (b, h0, h1) in enumerate(pipe.chunks):
+        _, c2, i2, _ = (t.cpu().numpy() for t in
+                        abatt.intermediates(pipe.ws[j], (1, h1 - h0, w.N, w.d), cfg))
+        for r in range((h1 - h0) * nQ):
+            a = set(i2[r, :c2[r]].tolist())
+            bb = set(i1[h0 * nQ + r, :c1[h0 * nQ + r]].tolist())
+            diff += len(a ^ bb)
+            tot += len(bb)
+    assert diff <= 0.001 * tot, (diff, tot)
+    got, ref = ho.float().numpy(), O1.float().cpu().numpy()
+    assert _rel_l2(got, ref) <= REL_L2
+    assert np.max(np.abs(got - ref)) <= MAX_ABS
