@@ -195,6 +195,33 @@ def cpu_baseline(w, Q, K, V, budget_s=15.0):
                       f"extrapolated x{w.rows / len(rows):.1f}"}
 
 
+def rank_plan(w, rank: int, world: int) -> dict:
+    """What rank `rank` of `world` computes (weak scaling, no collective on the
+    data path): batch elements [rank*B, (rank+1)*B) of a world*B-element
+    problem.  Its inputs are drawn with data seed w.seed + rank; its sampler
+    uses the global batch index (batch_offset) with the job's one Philox key."""
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside world {world}")
+    return {"batch_offset": rank * w.B, "data_seed": w.seed + rank, "philox_seed": w.seed}
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's time (every rank takes part; returns x when alone)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flop_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job dense-equivalent TFLOPS: the work of all ranks over the
+    slowest rank's time."""
+    return flop_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def main():
     args = parse()
     w = synth.WORKLOADS[args.workload]
@@ -218,11 +245,13 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    Qc, Kc, Vc = synth.generate(w)
+    plan = rank_plan(w, rank, world)
+    Qc, Kc, Vc = synth.generate(w.with_(seed=plan["data_seed"]))
     Q, K, V = Qc.to(dev), Kc.to(dev), Vc.to(dev)
     shape = w.shape
     cfg = abatt.Config(kv_block=w.Bk, clusters=w.clusters, kmeans_iters=w.iters,
-                       budget_bp=w.budget_bp, seed=w.seed)
+                       budget_bp=w.budget_bp, seed=plan["philox_seed"],
+                       batch_offset=plan["batch_offset"])
     rows, nK = w.rows, w.nK
     p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
     counts = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -265,11 +294,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
     sel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
     smp_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
     att_ms = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
@@ -302,7 +327,7 @@ def main():
 
     line = {
         "metric": METRIC,
-        "value": dense_flop * world / (ms_step * 1e-3) / 1e12,
+        "value": job_value(dense_flop, world, ms_step),
         "unit": "TFLOPS (dense-equivalent)",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -395,14 +420,10 @@ def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):
         step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
     dense = 4.0 * w.B * w.H * w.N * w.N * w.d
     nbytes = Qc.numel() * 2
-    return {"value": dense * world / (ms * 1e-3) / 1e12, "unit": "TFLOPS (dense-equivalent)",
+    return {"value": job_value(dense, world, ms), "unit": "TFLOPS (dense-equivalent)",
             "ms_per_step": ms, "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
             "steps": steps, "heads_per_chunk": pipe.hc, "device_status": pipe.status()}
 
