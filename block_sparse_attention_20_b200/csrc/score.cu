@@ -9,8 +9,8 @@
 // The centroid tile (fp16 of the pre-scaled fp32 centroids: 11 significant
 // bits, against 8 for bf16) stays in shared memory; 128-key fp16 tiles of K
 // stream through a 4-stage TMA ring; one warp issues tcgen05 MMAs
-// (kind::f16, fp32 accumulation) into a double-buffered 128x128 accumulator
-// in tensor memory; two epilogue warpgroups (one per accumulator buffer,
+// (kind::f16, fp32 accumulation) into four 128x128 accumulator buffers
+// in tensor memory; four epilogue warpgroups (one per accumulator buffer,
 // thread = centroid row) turn each tile into base-2 exponentials relative to
 // the row's running maximum and sum them per key block, two values per
 // packed fp32 instruction, with a fixed share of the exponentials on the FMA
@@ -28,7 +28,9 @@ namespace abatt {
 namespace {
 
 constexpr int kScoreStages = 4;
-constexpr int kScoreThreads = 320;  // warps 0-7 epilogue (2 warpgroups), 8 TMA, 9 MMA
+constexpr int kScoreEpi = 4;        // epilogue warpgroups = accumulator buffers in tensor memory
+constexpr int kScoreThreads = kScoreEpi * 128 + 64;  // + a TMA warp and an MMA warp
+constexpr int kWarpTma = kScoreEpi * 4, kWarpMma = kScoreEpi * 4 + 1;
 #define kNegInf (-__int_as_float(0x7f800000))
 // exponent pairs of every sixteen that the epilogue evaluates with the
 // FMA-pipe polynomial (the others use ex2)
@@ -91,10 +93,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     __shared__ __align__(8) uint64_t bar_a;
     __shared__ __align__(8) uint64_t bar_kfull[ST], bar_kempty[ST];
-    __shared__ __align__(8) uint64_t bar_sfull[2], bar_sempty[2];
+    __shared__ __align__(8) uint64_t bar_sfull[kScoreEpi], bar_sempty[kScoreEpi];
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
-    __shared__ float2 mz_s[128];
+    __shared__ float2 mz_s[kScoreEpi][128];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int mt = blockIdx.x, hd = blockIdx.y, chunk = blockIdx.z;
@@ -113,14 +115,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             mbar_init(&bar_kfull[s], 1);
             mbar_init(&bar_kempty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kScoreEpi; ++b) {
             mbar_init(&bar_sfull[b], 1);
             mbar_init(&bar_sempty[b], 4);
         }
         fence_barrier_init();
     }
-    if (warp == 9) {
-        tmem_alloc(&tmem_base_s, 256);
+    if (warp == kWarpMma) {
+        tmem_alloc(&tmem_base_s, 128 * kScoreEpi);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     int issued = 0;       // TMA role: K tiles issued
     int committed = -1;   // MMA role: last K tile whose MMAs were committed
 
-    if (warp == 8) {
+    if (warp == kWarpTma) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             tma_prefetch_desc(&maps.a);
@@ -147,7 +149,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 issued = i + 1;
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == kWarpMma) {
         // ------------------------------ MMA issuer --------------------------------
         // the whole warp follows the schedule (warp-uniform control flow and
         // descriptors); one elected lane issues each tcgen05 instruction
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             constexpr uint32_t idesc = idesc_f16(128, 128);
             const uint64_t da = sdesc_sw128(smem_u32(sA), 16, 1024);
             for (int i = 0; i < ntl; ++i) {
-                const int s = i % ST, buf = i & 1, use = i >> 1;
+                const int s = i % ST, buf = i % kScoreEpi, use = i / kScoreEpi;
                 if (!wait_all(&bar_kfull[s], (i / ST) & 1, 0x103)) break;
                 if (use > 0 && !wait_all(&bar_sempty[buf], (use - 1) & 1, 0x104)) break;
                 tc_fence_after();
@@ -177,6 +179,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------ epilogue ----------------------------------
+        // Warpgroup e takes the tiles i = e (mod kScoreEpi) from accumulator
+        // buffer e, 32 columns at a time in two passes (the tile maximum, then
+        // the exponentials), so a thread holds 32 scores, not 128.
         const int e = warp >> 2;        // accumulator buffer of this warpgroup
         const int wq = warp & 3;        // TMEM lane quarter
         const int rl = wq * 32 + lane;  // centroid row within the tile
@@ -184,38 +189,33 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const bool valid = grow < a.MC;
         const int64_t gr = (int64_t)hd * a.MC + grow;
         float m_run = kNegInf, Z = 0.0f;
-        for (int i = e; i < ntl; i += 2) {
-            const int kt = kt0 + i, use = i >> 1;
+        for (int i = e; i < ntl; i += kScoreEpi) {
+            const int kt = kt0 + i, use = i / kScoreEpi;
             if (!mbar_wait(&bar_sfull[e], use & 1, wc, 0x105)) break;
             tc_fence_after();
-            uint32_t v[4][32];
             const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + e * 128;
-            tmem_ld32(taddr + 0, v[0]);
-            tmem_ld32(taddr + 32, v[1]);
-            tmem_ld32(taddr + 64, v[2]);
-            tmem_ld32(taddr + 96, v[3]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_sempty[e]);
-
-            const int kbase = kt * 128;
-            const int nvalid = min(128, a.N - kbase);
-            if (nvalid < 128) {  // the sequence's last tile: keys past N count for nothing
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
+            const int nvalid = min(128, a.N - kt * 128);  // < 128 only on the sequence's last tile
+            auto load = [&](int q, uint32_t (&v)[32]) {
+                tmem_ld32(taddr + q * 32, v);
+                tmem_wait_ld();
+                if (nvalid < 128) {  // keys past N count for nothing
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
-                        if (q * 32 + c >= nvalid) v[q][c] = __float_as_uint(kNegInf);
-            }
-            // four independent max chains (one per 32-column load), then merged
+                        if (q * 32 + c >= nvalid) v[c] = __float_as_uint(kNegInf);
+                }
+            };
             float tq[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                tq[q] = kNegInf;
+                uint32_t v[32];
+                load(q, v);
+                float t0 = kNegInf, t1 = kNegInf;  // two independent max chains
 #pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    tq[q] = fmax3f(tq[q], __uint_as_float(v[q][c]), __uint_as_float(v[q][c + 1]));
+                for (int c = 0; c < 32; c += 4) {
+                    t0 = fmax3f(t0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+                    t1 = fmax3f(t1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                }
+                tq[q] = fmaxf(t0, t1);
             }
             const float tm = fmaxf(fmax3f(tq[0], tq[1], tq[2]), tq[3]);
             const float m_new = fmaxf(m_run, tm);
@@ -232,22 +232,28 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                 for (int u = 0; u < NA; ++u) acc[k][u] = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                load(q, v);
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const int col = q * 32 + c;
-                    const float2 x =
-                        __fadd2_rn(make_float2(__uint_as_float(v[q][c]), __uint_as_float(v[q][c + 1])), nm);
-                    float2 e;
+                    const float2 x = __fadd2_rn(make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), nm);
+                    float2 ex;
                     if (((col >> 1) & 15) < kScorePolyOf16) {
-                        e = exp2_poly2<4>(x);
+                        ex = exp2_poly2<4>(x);
                     } else {
-                        e.x = ex2_approx(x.x);
-                        e.y = ex2_approx(x.y);
+                        ex.x = ex2_approx(x.x);
+                        ex.y = ex2_approx(x.y);
                     }
                     float2 &s2 = acc[col / BK][(col >> 1) % NA];
-                    s2 = __fadd2_rn(s2, e);
+                    s2 = __fadd2_rn(s2, ex);
                 }
+            }
+            // the accumulator buffer is free for the tile after next
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_sempty[e]);
             float bs[BPT];
 #pragma unroll
             for (int k = 0; k < BPT; ++k) {
@@ -263,18 +269,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 a.mref[gr * a.nT + kt] = m_run;
             }
         }
-        if (e == 1) mz_s[rl] = make_float2(m_run, Z);
+        mz_s[e][rl] = make_float2(m_run, Z);
         tc_fence_before();
         __syncthreads();
         if (e == 0) {
-            const float2 o = mz_s[rl];
-            const float m = fmaxf(m_run, o.x);
-            const float z0 = (m_run == kNegInf) ? 0.0f : Z * ex2_approx(m_run - m);
-            const float z1 = (o.x == kNegInf) ? 0.0f : o.y * ex2_approx(o.x - m);
-            if (valid) a.mz[gr * a.nchunk + chunk] = make_float2(m, z0 + z1);
+            // merge the warpgroups' (max, sum) of this row
+            float m = kNegInf;
+#pragma unroll
+            for (int g = 0; g < kScoreEpi; ++g) m = fmaxf(m, mz_s[g][rl].x);
+            float z = 0.0f;
+#pragma unroll
+            for (int g = 0; g < kScoreEpi; ++g) {
+                const float2 o = mz_s[g][rl];
+                if (o.x != kNegInf) z += o.y * ex2_approx(o.x - m);
+            }
+            if (valid) a.mz[gr * a.nchunk + chunk] = make_float2(m, z);
         }
     }
-    if (warp >= 8) {
+    if (warp >= kWarpTma) {
         tc_fence_before();
         __syncthreads();  // pairs with the epilogue's barrier above
     }
@@ -282,14 +294,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     // ------------------------------ teardown --------------------------------------
     if (abort_s) {
         // drain copies and MMAs still in flight before shared/tensor memory go away
-        if (warp == 8 && lane == 0)
+        if (warp == kWarpTma && lane == 0)
             for (int t = issued - ST > 0 ? issued - ST : 0; t < issued; ++t) {
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(&bar_kfull[t % ST], (t / ST) & 1) &&
                        globaltimer_ns() - t0 < a.wait_ns) {
                 }
             }
-        if (warp == 9 && lane == 0 && committed >= 0) {
+        if (warp == kWarpMma && lane == 0 && committed >= 0) {
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&bar_kempty[committed % ST], (committed / ST) & 1) &&
                    globaltimer_ns() - t0 < a.wait_ns) {
@@ -297,9 +309,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     }
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 128 * kScoreEpi);
     }
 }
 
