@@ -170,7 +170,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                    umma_ss_w(d_tmem, da + off, kd + off, idesc, kk > 0);
+                    // after a buffer's first tile the epilogue leaves -m_ref in it:
+                    // accumulate onto it, so the product arrives as x - m_ref
+                    umma_ss_w(d_tmem, da + off, kd + off, idesc, (kk > 0 || use > 0) ? 1u : 0u);
                 }
                 umma_commit_w(&bar_kempty[s]);
                 umma_commit_w(&bar_sfull[buf]);
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int grow = mt * 128 + rl;
         const bool valid = grow < a.MC;
         const int64_t gr = (int64_t)hd * a.MC + grow;
-        float m_run = kNegInf, Z = 0.0f;
+        float m_run = kNegInf, Z = 0.0f;  // reference (base 2) and sum relative to it
         for (int i = e; i < ntl; i += kScoreEpi) {
             const int kt = kt0 + i, use = i / kScoreEpi;
             if (!mbar_wait(&bar_sfull[e], use & 1, wc, 0x105)) break;
@@ -204,64 +206,96 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         if (q * 32 + c >= nvalid) v[c] = __float_as_uint(kNegInf);
                 }
             };
-            float tq[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t v[32];
-                load(q, v);
-                float t0 = kNegInf, t1 = kNegInf;  // two independent max chains
-#pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    t0 = fmax3f(t0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
-                    t1 = fmax3f(t1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-                }
-                tq[q] = fmaxf(t0, t1);
-            }
-            const float tm = fmaxf(fmax3f(tq[0], tq[1], tq[2]), tq[3]);
-            const float m_new = fmaxf(m_run, tm);
-            const float alpha = (m_run == kNegInf) ? 0.0f : ex2_approx(m_run - m_new);
-            Z *= alpha;
-            m_run = m_new;
-            // 2^(x - m) two columns at a time; NA interleaved partial sums per
-            // block keep the add chains short when blocks are wide
+            // block sums of 2^(y - sub) over the tile, y the buffer's values
             constexpr int NA = BPT >= 8 ? 1 : 8 / BPT;
-            const float2 nm = make_float2(-m_run, -m_run);
-            float2 acc[BPT][NA];
+            float bs[BPT];
+            auto block_sums = [&](float sub) {
+                const float2 nm = make_float2(-sub, -sub);
+                float2 acc[BPT][NA];
 #pragma unroll
-            for (int k = 0; k < BPT; ++k)
+                for (int k = 0; k < BPT; ++k)
 #pragma unroll
-                for (int u = 0; u < NA; ++u) acc[k][u] = make_float2(0.0f, 0.0f);
+                    for (int u = 0; u < NA; ++u) acc[k][u] = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t v[32];
-                load(q, v);
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    load(q, v);
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const int col = q * 32 + c;
-                    const float2 x = __fadd2_rn(make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), nm);
-                    float2 ex;
-                    if (((col >> 1) & 15) < kScorePolyOf16) {
-                        ex = exp2_poly2<4>(x);
-                    } else {
-                        ex.x = ex2_approx(x.x);
-                        ex.y = ex2_approx(x.y);
+                    for (int c = 0; c < 32; c += 2) {
+                        const int col = q * 32 + c;
+                        float2 x = make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+                        if (sub != 0.0f) x = __fadd2_rn(x, nm);
+                        float2 ex;
+                        if (((col >> 1) & 15) < kScorePolyOf16) {
+                            // the polynomial is valid below 2^128: larger inputs land at
+                            // 2^100 and send the tile to the exact path below
+                            x.x = fminf(x.x, 100.0f);
+                            x.y = fminf(x.y, 100.0f);
+                            ex = exp2_poly2<4>(x);
+                        } else {
+                            ex.x = ex2_approx(x.x);
+                            ex.y = ex2_approx(x.y);
+                        }
+                        float2 &s2 = acc[col / BK][(col >> 1) % NA];
+                        s2 = __fadd2_rn(s2, ex);
                     }
-                    float2 &s2 = acc[col / BK][(col >> 1) % NA];
-                    s2 = __fadd2_rn(s2, ex);
                 }
+#pragma unroll
+                for (int k = 0; k < BPT; ++k) {
+                    float2 t2 = acc[k][0];
+#pragma unroll
+                    for (int u = 1; u < NA; ++u) t2 = __fadd2_rn(t2, acc[k][u]);
+                    bs[k] = t2.x + t2.y;
+                }
+            };
+            // exact path: the tile's own maximum mx of y (relative to the current
+            // reference, or absolute on the first tile) becomes part of the reference
+            auto exact = [&]() {
+                float tq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    load(q, v);
+                    float t0 = kNegInf, t1 = kNegInf;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        t0 = fmax3f(t0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+                        t1 = fmax3f(t1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                    }
+                    tq[q] = fmaxf(t0, t1);
+                }
+                const float mx = fmaxf(fmax3f(tq[0], tq[1], tq[2]), tq[3]);
+                const float base = (m_run == kNegInf) ? 0.0f : m_run;  // what y is relative to
+                const float m_new = fmaxf(m_run, base + mx);
+                const float alpha = (m_run == kNegInf) ? 0.0f : ex2_approx(m_run - m_new);
+                Z *= alpha;
+                m_run = m_new;
+                block_sums(m_new - base);
+            };
+            // first tile of this buffer (the MMA started from zero): exact path;
+            // later tiles: the buffer held -m_run, so y = x - m_run already, one
+            // pass of exponentials -- unless some row's scores outgrew its
+            // reference, then the warp redoes the tile with the exact maximum
+            // (correct for every row; tensor-memory loads stay warp-uniform)
+            bool redo = use == 0;
+            if (!redo) {
+                block_sums(0.0f);
+                float big = 0.0f;
+#pragma unroll
+                for (int k = 0; k < BPT; ++k) big = fmaxf(big, bs[k]);
+                redo = __any_sync(0xffffffffu, !(big < 0x1p80f));
             }
-            // the accumulator buffer is free for the tile after next
+            if (redo) exact();
+            // leave -m_run in the buffer for its next tile, then free it
+            if (i + kScoreEpi < ntl) {
+                const uint32_t nmr = __float_as_uint(m_run == kNegInf ? 0.0f : -m_run);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tmem_fill32(taddr + q * 32, nmr);
+                tmem_wait_st();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_sempty[e]);
-            float bs[BPT];
-#pragma unroll
-            for (int k = 0; k < BPT; ++k) {
-                float2 t2 = acc[k][0];
-#pragma unroll
-                for (int u = 1; u < NA; ++u) t2 = __fadd2_rn(t2, acc[k][u]);
-                bs[k] = t2.x + t2.y;
-            }
 #pragma unroll
             for (int k = 0; k < BPT; ++k) Z += bs[k];
             if (valid) {

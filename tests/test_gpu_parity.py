@@ -296,6 +296,22 @@ def test_select_d128_ragged(Bk, C):
     _select_check(Q, K, w.shape, C, 5, Bk)
 
 
+def test_select_scores_that_grow_along_the_keys():
+    # keys along one direction with norms growing 1x -> 20x over the sequence:
+    # every centroid's logits rise by ~200 (base 2) from the first key tile to
+    # the last, past the reference the scoring epilogue starts from, so later
+    # tiles take its exact (re-referenced) path
+    N, d = 2048, 64
+    rng = np.random.default_rng(5)
+    u = rng.standard_normal(d)
+    g = np.linspace(1.0, 20.0, N)
+    q = np.tile(u, (N, 1)) + 0.05 * rng.standard_normal((N, d))
+    k = g[:, None] * u[None, :] + 0.05 * rng.standard_normal((N, d))
+    Q = torch.from_numpy(q[None, None]).to(torch.bfloat16)
+    K = torch.from_numpy(k[None, None]).to(torch.bfloat16)
+    _select_check(Q, K, (1, 1, N, d), 2, 1, 16)
+
+
 # ------------------------------------------------------------------------- end to end
 
 def _forward_check(w, rows_check, heads=None):
