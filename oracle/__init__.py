@@ -56,6 +56,7 @@ def _load():
         lib.orc_budget_blocks.argtypes = [i32, i32]
         lib.orc_budget_blocks.restype = i64
         lib.orc_inclusion.argtypes = [P, i32, i64, P, P, P, P, P]
+        lib.orc_topk.argtypes = [P, i64, i32, i32, i32, i32, P, P, P]
         lib.orc_sample.argtypes = [P, i32, i32, i32, i32, i32, P, i64, i32, u64, i32, i32,
                                    P, P, P, P]
         lib.orc_ht_attention.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, i64,
@@ -195,6 +196,24 @@ def sample(p, shape, rows, budget_bp, seed, Bq=128, Bk=16, capacity=None, nthrea
                                    int(seed) & (2**64 - 1), cap, nthreads or default_threads(),
                                    _ptr(counts), _ptr(idx), _ptr(logw), _ptr(amb)), "sample")
     return counts, idx, logw, amb, bool(rc == 1)
+
+
+def topk(p, budget_bp, capacity=None, nthreads=None):
+    """O4': top-M truncation of fp32 probability rows p [nrows, nK]: the M
+    largest (48-bit fixed point, ties to the lower index), ascending, log-weight
+    0.  Returns counts [nrows], idx [nrows, cap], logw fp32 [nrows, cap],
+    overflow flag."""
+    p = np.ascontiguousarray(np.asarray(p, dtype=np.float32))
+    nrows, nK = p.shape
+    cap = nK if capacity is None else int(capacity)
+    counts = np.zeros(nrows, dtype=np.int32)
+    idx = np.full((nrows, cap), -1, dtype=np.int32)
+    logw = np.zeros((nrows, cap), dtype=np.float32)
+    rc = _load().orc_topk(_ptr(p), nrows, nK, int(budget_bp), cap, nthreads or default_threads(),
+                          _ptr(counts), _ptr(idx), _ptr(logw))
+    if rc < 0:
+        raise RuntimeError(f"orc_topk failed ({rc})")
+    return counts, idx, logw, bool(rc == 1)
 
 
 def ht_attention(Q, K, V, shape, rows, counts, idx, logw, Bq=128, Bk=16, scale=None,

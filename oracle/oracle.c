@@ -655,6 +655,79 @@ int orc_sample(const float *p, int B, int H, int N, int Bq, int Bk,
 }
 
 /* ------------------------------------------------------------------------ */
+/* O4' Top-M truncation, the baseline the abstract contrasts with SIP: keep  */
+/* the M blocks with the largest estimate (ranked on the same 48-bit fixed   */
+/* point as the sampler, ties to the lower block index), ascending, each     */
+/* with log-weight 0 (no reweighting).  M >= nK keeps every block.          */
+/* ------------------------------------------------------------------------ */
+
+typedef struct { int64_t P; int32_t b; } rank_t;
+
+static int rank_cmp(const void *x, const void *y)
+{
+    const rank_t *a = (const rank_t *)x, *c = (const rank_t *)y;
+    if (a->P != c->P) return a->P > c->P ? -1 : 1;  /* larger estimate first */
+    return a->b < c->b ? -1 : (a->b > c->b);        /* then lower index */
+}
+
+static int topk_row(const float *p, int nK, int budget_bp, int capacity, int32_t *count,
+                    int32_t *idx, float *logw, int *overflow)
+{
+    const int64_t M = orc_budget_blocks(budget_bp, nK);
+    const int keep = M >= nK ? nK : (int)M;
+    rank_t *r = (rank_t *)malloc(sizeof(rank_t) * (size_t)nK);
+    uint8_t *take = (uint8_t *)calloc((size_t)nK, 1);
+    if (!r || !take) { free(r); free(take); return -3; }
+    for (int b = 0; b < nK; ++b) { r[b].P = to_fixed(p[b]); r[b].b = b; }
+    qsort(r, (size_t)nK, sizeof(rank_t), rank_cmp);
+    for (int k = 0; k < keep; ++k) take[r[k].b] = 1;
+    int n = 0;
+    *overflow = 0;
+    for (int b = 0; b < nK; ++b) {
+        if (!take[b]) continue;
+        if (n < capacity) { idx[n] = b; logw[n] = 0.0f; ++n; }
+        else *overflow = 1;
+    }
+    *count = n;
+    free(r); free(take);
+    return 0;
+}
+
+typedef struct {
+    const float *p;
+    int nK, budget_bp, capacity;
+    int32_t *counts, *idx;
+    float *logw;
+    int bad, overflow;
+} topk_ctx;
+
+static void topk_job(void *vctx, int64_t k)
+{
+    topk_ctx *c = (topk_ctx *)vctx;
+    int of = 0;
+    size_t o = (size_t)k * c->capacity;
+    if (topk_row(c->p + (size_t)k * c->nK, c->nK, c->budget_bp, c->capacity, c->counts + k,
+                 c->idx + o, c->logw + o, &of))
+        c->bad = 1;
+    if (of) __atomic_store_n(&c->overflow, 1, __ATOMIC_RELAXED);
+}
+
+/* p is [nrows][nK].  Returns 1 if some row kept more blocks than `capacity`. */
+int orc_topk(const float *p, int64_t nrows, int nK, int budget_bp, int capacity, int nthreads,
+             int32_t *counts, int32_t *idx, float *logw)
+{
+    if (!p || !counts || !idx || !logw || nK <= 0 || nK > 32767 || capacity < 0 || budget_bp < 0)
+        return -1;
+    topk_ctx c;
+    memset(&c, 0, sizeof c);
+    c.p = p; c.nK = nK; c.budget_bp = budget_bp; c.capacity = capacity;
+    c.counts = counts; c.idx = idx; c.logw = logw;
+    parallel_for(nrows, nthreads, topk_job, &c);
+    if (c.bad) return -2;
+    return c.overflow ? 1 : 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* O5  attention restricted to the drawn blocks, each logit shifted by its   */
 /* block's log-weight -ln(pi_b) (multiplying its exponential by 1/pi_b).     */
 /* Numerator and denominator are then Horvitz-Thompson estimates of the      */
