@@ -51,6 +51,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (s->B <= 0 || s->H <= 0 || s->N <= 0 || s->d <= 0) return ABATT_ERR_INVALID_ARG;
     if (c->budget_bp < 0 || !(c->scale > 0.0f) || !isfinite(c->scale)) return ABATT_ERR_INVALID_ARG;
     if (c->batch_offset < 0 || c->head_offset < 0) return ABATT_ERR_INVALID_ARG;
+    if (c->selection != ABATT_SELECT_SIP && c->selection != ABATT_SELECT_TOPK) return ABATT_ERR_INVALID_ARG;
     if (s->d != 64 && s->d != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->q_block != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->kv_block != 16 && c->kv_block != 32 && c->kv_block != 64 && c->kv_block != 128)
@@ -69,6 +70,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (g->rows >= (int64_t(1) << 31) || g->heads > 65535) return ABATT_ERR_UNSUPPORTED;
     if ((int64_t)s->N * s->d * g->heads >= (int64_t(1) << 40)) return ABATT_ERR_UNSUPPORTED;
     g->M = ((int64_t)c->budget_bp * g->nK + 5000) / 10000;
+    if (c->selection == ABATT_SELECT_TOPK && g->nK > 10240) return ABATT_ERR_UNSUPPORTED;
     return ABATT_OK;
 }
 
@@ -242,6 +244,7 @@ abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, 
     SampleArgs a;
     a.p = p; a.rows = g.rows; a.nK = g.nK; a.nK_pad = (g.nK + 3) & ~3; a.nQ = g.nQ; a.H = g.H;
     a.M = g.M;
+    a.topk = cfg->selection == ABATT_SELECT_TOPK ? 1 : 0;
     a.b_off = (uint32_t)cfg->batch_offset;
     a.h_off = (uint32_t)cfg->head_offset;
     a.key0 = (uint32_t)(cfg->seed & 0xffffffffu);

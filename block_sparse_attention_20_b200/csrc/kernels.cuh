@@ -67,6 +67,7 @@ struct SampleArgs {
     int nK, nK_pad, nQ, H;
     int64_t M;
     uint32_t b_off, h_off;  // global index of the first batch element / head (Philox counter)
+    int topk;               // 1: keep the M largest estimates (weight 1) instead of drawing
     uint32_t key0, key1;
     int capacity;
     int32_t *counts, *idx;

@@ -241,6 +241,9 @@ __global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
     __shared__ int32_t red_c[NW];
     __shared__ int32_t wtot[NW];
     __shared__ uint32_t sat_s[NT];  // saturation mask of each thread's run
+    __shared__ int32_t hist_s[128];  // top-M: digit histogram of the radix select
+    __shared__ int64_t sel_prefix_s;
+    __shared__ int32_t sel_k_s;
     const int nK = a.nK;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b0 = tid * PER;
@@ -279,9 +282,92 @@ __global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
         const int nmine = max(0, min(PER, nK - b0));
         const uint32_t valid = nmine >= 32 ? 0xffffffffu : ((1u << nmine) - 1u);
 
-        // ---- inclusion probabilities: exact water-filling (as in the shared-memory kernel)
-        uint32_t sat = 0;
+        uint32_t sat = 0, take = 0;
         int64_t R = a.M, T = 0;
+        if (a.topk) {
+            // ---- top-M truncation: the M largest weights, ties to the lower index.
+            // Radix select of the M-th largest key, seven 7-bit digits from the
+            // top (keys are < 2^49), then the ties admitted in index order.
+            if (a.M >= nK) {
+                take = valid;
+            } else if (a.M > 0) {
+                int64_t prefix = 0, mask = 0;
+                int k = (int)a.M;  // rank still to find among the candidates, 1 = largest
+                for (int dgt = 6; dgt >= 0; --dgt) {
+                    const int sh = 7 * dgt;
+                    if (tid < 128) hist_s[tid] = 0;
+                    __syncthreads();
+#pragma unroll
+                    for (int q = 0; q < PER; ++q)
+                        if (((valid >> q) & 1u) && (P[q] & mask) == prefix)
+                            atomicAdd(&hist_s[(int)((P[q] >> sh) & 127)], 1);
+                    __syncthreads();
+                    if (warp == 0) {
+                        // lane l holds bins 4l..4l+3; counts at or above each bin by a
+                        // suffix scan over the lanes, from the largest digit down
+                        int c[4], sum = 0;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) { c[u] = hist_s[4 * lane + u]; sum += c[u]; }
+                        int suf = sum;  // inclusive suffix over lanes l..31
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_down_sync(0xffffffffu, suf, o);
+                            if (lane + o < 32) suf += y;
+                        }
+                        int above = suf - sum;  // keys in bins of higher lanes
+                        int found = -1, above_found = 0;
+#pragma unroll
+                        for (int u = 3; u >= 0; --u) {
+                            if (found < 0 && above < k && above + c[u] >= k) {
+                                found = 4 * lane + u;
+                                above_found = above;
+                            }
+                            above += c[u];
+                        }
+                        const uint32_t who = __ballot_sync(0xffffffffu, found >= 0);
+                        const int src = __ffs(who) - 1;
+                        const int v = __shfl_sync(0xffffffffu, found, src);
+                        const int ab = __shfl_sync(0xffffffffu, above_found, src);
+                        if (lane == 0) {
+                            sel_prefix_s = prefix | ((int64_t)v << sh);
+                            sel_k_s = k - ab;
+                        }
+                    }
+                    __syncthreads();
+                    prefix = sel_prefix_s;
+                    k = sel_k_s;
+                    mask |= (int64_t)127 << sh;
+                    __syncthreads();  // hist_s and the selection are reused next digit
+                }
+                // prefix is the M-th largest key; k of the keys equal to it are kept,
+                // the first k by index: an exclusive scan of the per-thread tie counts
+                uint32_t ties = 0;
+#pragma unroll
+                for (int q = 0; q < PER; ++q) {
+                    if (!((valid >> q) & 1u)) continue;
+                    if (P[q] > prefix) take |= 1u << q;
+                    else if (P[q] == prefix) ties |= 1u << q;
+                }
+                const int tc = __popc(ties);
+                int x = tc;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                if (lane == 31) wtot[warp] = x;
+                __syncthreads();
+                int before = x - tc;
+#pragma unroll
+                for (int q = 0; q < NW; ++q) before += q < warp ? wtot[q] : 0;
+                __syncthreads();  // wtot is reused by the compaction
+#pragma unroll
+                for (int q = 0; q < PER; ++q)
+                    if (((ties >> q) & 1u) && before++ < k) take |= 1u << q;
+            }
+            sat = take;  // kept blocks carry log-weight 0
+        } else {
+        // ---- inclusion probabilities: exact water-filling (as in the shared-memory kernel)
         if (a.M >= nK) {
             sat = valid;
             R = 0;
@@ -337,7 +423,6 @@ __global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
         sat &= valid;
 
         // ---- draws: group g = tid*G + u gives blocks 4g..4g+3 ----------------
-        uint32_t take = 0;
 #pragma unroll
         for (int u = 0; u < G; ++u) {
             const int g = tid * G + u;
@@ -357,6 +442,7 @@ __global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
                 }
             }
         }
+        }  // SIP
         // ---- ordered compaction: exclusive scan of the per-thread counts -------
         const int cnt = __popc(take);
         int x = cnt;

@@ -67,6 +67,15 @@ typedef struct abatt_shape {
     int d; /* head dimension */
 } abatt_shape;
 
+/* How abatt_sample (and abatt_forward) turn block probabilities into lists.
+   SIP: the abstract's sampler -- a Poisson draw with pi_b = min(1, c*p_b),
+        sum pi = M, each drawn block weighted by 1/pi_b (log-weight -ln pi_b).
+   TOPK: the truncating baseline the abstract contrasts it with -- the M blocks
+        with the largest estimate (ranked on the same 48-bit fixed point, ties to
+        the lower index), each with log-weight 0.  Needs nK <= 10240
+        (ABATT_ERR_UNSUPPORTED otherwise). */
+enum { ABATT_SELECT_SIP = 0, ABATT_SELECT_TOPK = 1 };
+
 typedef struct abatt_config {
     int q_block;        /* Bq: queries per query block (128) */
     int kv_block;       /* Bk: keys per key/value block (16 by default) */
@@ -79,6 +88,7 @@ typedef struct abatt_config {
     uint64_t seed;      /* Philox key for the draws */
     int batch_offset;   /* global index of this call's first batch element (0 for a whole tensor) */
     int head_offset;    /* global index of this call's first head (0 for a whole tensor) */
+    int selection;      /* ABATT_SELECT_SIP (0, the method) or ABATT_SELECT_TOPK (1) */
     /* The sampler's Philox counter uses the global indices (beta + batch_offset,
        h + head_offset), so a call over a slice of the batches or heads of a
        larger problem draws exactly the blocks that one call over the whole

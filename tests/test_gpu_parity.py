@@ -93,6 +93,33 @@ def test_sample_bit_exact(nK, Bk, bp, conc):
     _check_lists_exact(c.cpu().numpy(), i.cpu().numpy(), lw.cpu().numpy(), oc, oi, ol, oamb)
 
 
+@pytest.mark.parametrize("nK,bp,coarse", [(256, 1000, False), (4725, 800, True), (700, 2500, True),
+                                           (1500, 1200, False), (2900, 900, True), (5500, 700, False),
+                                           (9001, 1100, True), (63, 10000, False), (100, 0, False),
+                                           (1, 1000, False), (3, 5000, True)])
+def test_sample_topk_bit_exact(nK, bp, coarse):
+    Bk = 16
+    N = nK * Bk - (Bk // 2 if nK > 1 else 0)
+    shape = (1, 2, N, 64)
+    rows = _rows_of(shape)
+    p = synth.random_probs(len(rows), nK, 500 + nK, 0.2)
+    if coarse:  # many exact ties at the cut
+        p = (np.round(p * 64) / 64).astype(np.float32)
+    p[0] = 0  # all ties
+    if len(rows) > 2:
+        p[1, :] = np.float32(1.0 / nK)
+        p[2, 0] = np.nan
+    cfg = abatt.Config(kv_block=Bk, budget_bp=bp, selection=abatt.SELECT_TOPK)
+    c, i, lw, ws = abatt.sample(torch.from_numpy(p).cuda(), shape, cfg)
+    assert abatt.read_status(ws) == 0
+    oc, oi, ol, _ = oracle.topk(p, bp)
+    c, i, lw = c.cpu().numpy(), i.cpu().numpy(), lw.cpu().numpy()
+    assert np.array_equal(c, oc)
+    for r in range(len(rows)):
+        assert np.array_equal(i[r, :c[r]], oi[r, :c[r]]), r
+        assert np.all(lw[r, :c[r]] == 0)
+
+
 def test_sample_capacity_overflow_flags_and_truncates():
     nK, Bk = 512, 16
     shape = (1, 1, nK * Bk, 64)
@@ -413,3 +440,32 @@ def test_host_pipeline_matches_one_forward():
     got, ref = ho.float().numpy(), O1.float().cpu().numpy()
     assert _rel_l2(got, ref) <= REL_L2
     assert np.max(np.abs(got - ref)) <= MAX_ABS
+
+
+def test_forward_topk_tiny():
+    # the truncating baseline end to end: lists are the M largest of the
+    # kernel's own estimates, attention runs on them with weight 1
+    w = synth.TINY
+    Q, K, V = synth.generate(w)
+    shape = w.shape
+    cfg = cfg_of(w, selection=abatt.SELECT_TOPK)
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, shape, cfg), dtype=torch.uint8,
+                     device="cuda")
+    O = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg, workspace=ws)
+    torch.cuda.synchronize()
+    assert abatt.read_status(ws) == 0
+    p, counts, idx, logw = (t.cpu().numpy() for t in abatt.intermediates(ws, shape, cfg))
+    oc, oi, _, _ = oracle.topk(p, w.budget_bp)
+    assert np.array_equal(counts, oc)
+    rows = _rows_of(shape)
+    for r in rows:
+        assert np.array_equal(idx[r, :counts[r]], oi[r, :oc[r]])
+        assert np.all(logw[r, :counts[r]] == 0)
+    o5, _ = oracle.ht_attention(Q, K, V, shape, rows, counts, idx, logw, Bk=w.Bk)
+    Oc = O.float().cpu().numpy()
+    got = np.zeros_like(o5)
+    for r in rows:
+        h, q = divmod(int(r), w.nQ)
+        got[r] = Oc[0, h, q * 128:(q + 1) * 128]
+    assert _rel_l2(got, o5) <= REL_L2
+    assert np.max(np.abs(got - o5)) <= MAX_ABS
