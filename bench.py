@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-keep-all", action="store_true", help="skip the keep-all attention timing")
     ap.add_argument("--e2e-heads", type=int, default=2, help="heads per chunk of the host pipeline")
+    ap.add_argument("--selection", default="sip", choices=["sip", "topk"],
+                    help="sip: the method's draw; topk: the truncating baseline")
     return ap.parse_args()
 
 
@@ -251,7 +253,8 @@ def main():
     shape = w.shape
     cfg = abatt.Config(kv_block=w.Bk, clusters=w.clusters, kmeans_iters=w.iters,
                        budget_bp=w.budget_bp, seed=plan["philox_seed"],
-                       batch_offset=plan["batch_offset"])
+                       batch_offset=plan["batch_offset"],
+                       selection=abatt.SELECT_TOPK if args.selection == "topk" else abatt.SELECT_SIP)
     rows, nK = w.rows, w.nK
     p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
     counts = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -334,7 +337,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters,
-                   "kmeans_iters": w.iters, "per_rank": "one batch element per GPU",
+                   "kmeans_iters": w.iters, "selection": args.selection,
+                   "per_rank": "one batch element per GPU",
                    "l2": "inputs (Q,K,V 2.3 GB) exceed the 126 MB L2; no flush"},
         "stages_ms": {"select": sel_ms, "sample": smp_ms, "attention": att_ms},
         "attention_ms": att_ms,
