@@ -51,7 +51,7 @@ def _load():
         lib.orc_philox4x32_10.restype = None
         lib.orc_dense_attention.argtypes = [P, P, P, i32, i32, i32, i32, i32, f64, P, i64, i32, P, P]
         lib.orc_kmeans.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, i64, i32, P, P, P, P]
-        lib.orc_block_probs.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f64,
+        lib.orc_block_probs.argtypes = [P, P, i32, i32, i32, i32, i32, i32, i32, i32, f64, i32,
                                         P, i64, i32, P, P]
         lib.orc_budget_blocks.argtypes = [i32, i32]
         lib.orc_budget_blocks.restype = i64
@@ -142,8 +142,12 @@ def kmeans(Q, shape, rows, C, iters, Bq=128, nthreads=None, want_trace=False):
     return (cent, cnt, asg, trace) if want_trace else (cent, cnt, asg)
 
 
-def block_probs(Q, K, shape, rows, C, iters, Bq=128, Bk=16, scale=None, nthreads=None):
-    """O3: IBCS block probabilities. Returns (p float64, p fp32) [nrows, nK]."""
+def block_probs(Q, K, shape, rows, C, iters, Bq=128, Bk=16, scale=None, nthreads=None,
+                coarse=False):
+    """O3: IBCS block probabilities. Returns (p float64, p fp32) [nrows, nK].
+
+    coarse=True: O3', each key block scored once through its mean key, its
+    share n_b * exp(scale * c.kbar_b) normalised over the blocks."""
     B, H, N, d = shape
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     nK = -(-N // Bk)
@@ -151,7 +155,7 @@ def block_probs(Q, K, shape, rows, C, iters, Bq=128, Bk=16, scale=None, nthreads
     p64 = np.zeros((len(r), nK), dtype=np.float64)
     p32 = np.zeros((len(r), nK), dtype=np.float32)
     _check(_load().orc_block_probs(_ptr(_bits(Q)), _ptr(_bits(K)), B, H, N, d, Bq, Bk, C, iters,
-                                   scale, _ptr(r), len(r), nthreads or default_threads(),
+                                   scale, int(bool(coarse)), _ptr(r), len(r), nthreads or default_threads(),
                                    _ptr(p64), _ptr(p32)), "block_probs")
     return p64, p32
 

@@ -388,8 +388,15 @@ int orc_kmeans(const uint16_t *Q, int B, int H, int N, int d, int Bq, int C, int
 /* importance from the clustered queries.                                    */
 /* ------------------------------------------------------------------------ */
 
+/* Coarse variant (the abstract's other contrast: blocks "scored from coarse */
+/* summaries"): each key block b is scored once through its mean key kbar_b  */
+/* (the mean of its valid keys), with the block's share of the softmax       */
+/* taken as n_b * exp(scale * c.kbar_b) normalised over the blocks (n_b =    */
+/* valid keys of b) -- the per-key rule above applied to keys replaced by    */
+/* their block means.  Same centroids and weights.                           */
+
 static int block_probs_row(const uint16_t *Q, const uint16_t *K, const geom_t *g,
-                           int beta, int h, int i, int C, int iters, double scale,
+                           int beta, int h, int i, int C, int iters, double scale, int coarse,
                            double *p /*[nK]*/)
 {
     const int d = g->d, N = g->N, nK = g->nK;
@@ -404,6 +411,38 @@ static int block_probs_row(const uint16_t *Q, const uint16_t *K, const geom_t *g
     }
     int rc = kmeans_block(Q, g, beta, h, i, C, iters, cent, count, assign, NULL);
     for (int b = 0; b < nK; ++b) p[b] = 0.0;
+    if (coarse && rc == 0) {
+        double *kbar = (double *)malloc(sizeof(double) * (size_t)nK * d);
+        if (!kbar) rc = -3;
+        for (int b = 0; rc == 0 && b < nK; ++b) {
+            const int nb = keys_in_block(g, b);
+            for (int x = 0; x < d; ++x) {
+                double sum = 0.0;
+                for (int u = 0; u < nb; ++u) sum += bf16_to_f64(tok(K, g, beta, h, b * g->Bk + u)[x]);
+                kbar[(size_t)b * d + x] = sum / nb;
+            }
+        }
+        for (int j = 0; rc == 0 && j < C; ++j) {
+            if (count[j] == 0) continue;
+            const double w = (double)count[j] / (double)n;
+            double m = -INFINITY;
+            for (int b = 0; b < nK; ++b) {
+                double dot = 0.0;
+                for (int x = 0; x < d; ++x) dot += cent[(size_t)j * d + x] * kbar[(size_t)b * d + x];
+                z[b] = scale * dot + log((double)keys_in_block(g, b));
+                if (z[b] > m) m = z[b];
+            }
+            double Z = 0.0;
+            for (int b = 0; b < nK; ++b) {
+                z[b] = exp(z[b] - m);
+                Z += z[b];
+            }
+            for (int b = 0; b < nK; ++b) p[b] += w * (z[b] / Z);
+        }
+        free(kbar);
+        free(cent); free(count); free(assign); free(z);
+        return rc;
+    }
     for (int j = 0; rc == 0 && j < C; ++j) {
         if (count[j] == 0) continue;
         const double w = (double)count[j] / (double)n;
@@ -433,6 +472,7 @@ typedef struct {
     geom_t g;
     int C, iters;
     double scale;
+    int coarse;
     const int64_t *rows;
     double *p64;
     float *p32;
@@ -445,7 +485,7 @@ static void bp_row(void *vctx, int64_t k)
     int beta, h, i;
     if (decode_row(&c->g, c->rows[k], &beta, &h, &i)) { c->bad = 1; return; }
     double *p = c->p64 + (size_t)k * c->g.nK;
-    if (block_probs_row(c->Q, c->K, &c->g, beta, h, i, c->C, c->iters, c->scale, p)) {
+    if (block_probs_row(c->Q, c->K, &c->g, beta, h, i, c->C, c->iters, c->scale, c->coarse, p)) {
         c->bad = 1;
         return;
     }
@@ -454,7 +494,7 @@ static void bp_row(void *vctx, int64_t k)
 }
 
 int orc_block_probs(const uint16_t *Q, const uint16_t *K, int B, int H, int N, int d,
-                    int Bq, int Bk, int C, int iters, double scale,
+                    int Bq, int Bk, int C, int iters, double scale, int coarse,
                     const int64_t *rows, int64_t nrows, int nthreads,
                     double *p64, float *p32)
 {
@@ -462,7 +502,7 @@ int orc_block_probs(const uint16_t *Q, const uint16_t *K, int B, int H, int N, i
     memset(&c, 0, sizeof c);
     if (make_geom(&c.g, B, H, N, d, Bq, Bk)) return -1;
     if (C <= 0 || C > Bq || iters < 0 || !Q || !K || !rows || !p64) return -1;
-    c.Q = Q; c.K = K; c.C = C; c.iters = iters; c.scale = scale; c.rows = rows;
+    c.Q = Q; c.K = K; c.C = C; c.iters = iters; c.scale = scale; c.coarse = coarse; c.rows = rows;
     c.p64 = p64; c.p32 = p32;
     parallel_for(nrows, nthreads, bp_row, &c);
     return c.bad ? -2 : 0;
@@ -879,7 +919,7 @@ static void fwd_row(void *vctx, int64_t k)
     float *p32 = c->p32 + (size_t)k * nK;
     int32_t *idx = c->idx + (size_t)k * nK;
     float *logw = c->logw + (size_t)k * nK;
-    if (block_probs_row(c->Q, c->K, g, beta, h, i, c->C, c->iters, c->scale, p)) {
+    if (block_probs_row(c->Q, c->K, g, beta, h, i, c->C, c->iters, c->scale, 0, p)) {
         c->bad = 1;
     } else {
         for (int b = 0; b < nK; ++b) p32[b] = (float)p[b];
