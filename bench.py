@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--e2e-heads", type=int, default=2, help="heads per chunk of the host pipeline")
     ap.add_argument("--selection", default="sip", choices=["sip", "topk"],
                     help="sip: the method's draw; topk: the truncating baseline")
+    ap.add_argument("--scoring", default="keys", choices=["keys", "block-means"],
+                    help="keys: every key scored (the method); block-means: the coarse baseline")
     return ap.parse_args()
 
 
@@ -254,7 +256,9 @@ def main():
     cfg = abatt.Config(kv_block=w.Bk, clusters=w.clusters, kmeans_iters=w.iters,
                        budget_bp=w.budget_bp, seed=plan["philox_seed"],
                        batch_offset=plan["batch_offset"],
-                       selection=abatt.SELECT_TOPK if args.selection == "topk" else abatt.SELECT_SIP)
+                       selection=abatt.SELECT_TOPK if args.selection == "topk" else abatt.SELECT_SIP,
+                       scoring=(abatt.SCORE_BLOCK_MEANS if args.scoring == "block-means"
+                                else abatt.SCORE_KEYS))
     rows, nK = w.rows, w.nK
     p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
     counts = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -338,6 +342,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters,
                    "kmeans_iters": w.iters, "selection": args.selection,
+                   "scoring": args.scoring,
                    "per_rank": "one batch element per GPU",
                    "l2": "inputs (Q,K,V 2.3 GB) exceed the 126 MB L2; no flush"},
         "stages_ms": {"select": sel_ms, "sample": smp_ms, "attention": att_ms},

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libabatt.so")
 
 CALL_SELECT, CALL_SAMPLE, CALL_ATTENTION, CALL_FORWARD = 0, 1, 2, 3
 SELECT_SIP, SELECT_TOPK = 0, 1
+SCORE_KEYS, SCORE_BLOCK_MEANS = 0, 1
 DEVFLAG_CAPACITY, DEVFLAG_TIMEOUT, DEVFLAG_BADLIST = 0x1, 0x2, 0x4
 
 # Every symbol declared in include/abatt.h.
@@ -46,7 +47,7 @@ class _Config(ctypes.Structure):
                 ("kmeans_iters", ctypes.c_int), ("budget_bp", ctypes.c_int),
                 ("scale", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("batch_offset", ctypes.c_int), ("head_offset", ctypes.c_int),
-                ("selection", ctypes.c_int)]
+                ("selection", ctypes.c_int), ("scoring", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -63,12 +64,13 @@ class Config:
     batch_offset: int = 0  # global index of the call's first batch element
     head_offset: int = 0   # global index of the call's first head
     selection: int = 0     # SELECT_SIP (the method) or SELECT_TOPK (truncating baseline)
+    scoring: int = 0       # SCORE_KEYS (the method as read) or SCORE_BLOCK_MEANS (coarse baseline)
 
     def _c(self, d: int) -> _Config:
         s = self.scale if self.scale is not None else 1.0 / math.sqrt(d)
         return _Config(self.q_block, self.kv_block, self.clusters, self.kmeans_iters,
                        self.budget_bp, s, self.seed & (2**64 - 1), self.batch_offset, self.head_offset,
-                       self.selection)
+                       self.selection, self.scoring)
 
 
 _lock = threading.Lock()

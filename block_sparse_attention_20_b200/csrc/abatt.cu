@@ -3,6 +3,7 @@
 // sequence of each call.  No allocation, no synchronisation except in
 // abatt_read_status.
 #include <math.h>
+#include <algorithm>
 #include <mutex>
 #include <string.h>
 
@@ -17,6 +18,7 @@ constexpr float kLog2eF = 1.4426950408889634f;
 
 struct Geom {
     int B, H, N, d, Bq, Bk, C, I, nQ, nK, nT, ldr;
+    int nTc;  // coarse scoring: tiles of 128 key blocks; r rows then hold nTc*128 values
     int64_t rows, heads, M;
 };
 
@@ -52,6 +54,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (c->budget_bp < 0 || !(c->scale > 0.0f) || !isfinite(c->scale)) return ABATT_ERR_INVALID_ARG;
     if (c->batch_offset < 0 || c->head_offset < 0) return ABATT_ERR_INVALID_ARG;
     if (c->selection != ABATT_SELECT_SIP && c->selection != ABATT_SELECT_TOPK) return ABATT_ERR_INVALID_ARG;
+    if (c->scoring != ABATT_SCORE_KEYS && c->scoring != ABATT_SCORE_BLOCK_MEANS) return ABATT_ERR_INVALID_ARG;
     if (s->d != 64 && s->d != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->q_block != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->kv_block != 16 && c->kv_block != 32 && c->kv_block != 64 && c->kv_block != 128)
@@ -64,6 +67,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     g->nK = (s->N + g->Bk - 1) / g->Bk;
     g->nT = (s->N + 127) / 128;
     g->ldr = g->nT * (128 / g->Bk);
+    g->nTc = (g->nK + 127) / 128;
     g->heads = (int64_t)s->B * s->H;
     g->rows = g->heads * g->nQ;
     if (g->nK > 32767) return ABATT_ERR_UNSUPPORTED;
@@ -95,8 +99,9 @@ Layout layout(abatt_call call, const Geom &g) {
         L.cent16 = off;  off = align256(off + crow * g.d * 2);
         L.k16 = off;     off = align256(off + (size_t)g.heads * g.N * g.d * 2);
         L.weight = off;  off = align256(off + crow * 4);
-        L.r = off;       off = align256(off + crow * g.ldr * 4);
-        L.mref = off;    off = align256(off + crow * g.nT * 4);
+        const size_t ldr = std::max((size_t)g.ldr, (size_t)g.nTc * 128);  // either scoring rule
+        L.r = off;       off = align256(off + crow * ldr * 4);
+        L.mref = off;    off = align256(off + crow * std::max(g.nT, g.nTc) * 4);
         L.mz = off;      off = align256(off + crow * 8 * kMaxScoreChunks);
     }
     if (call == ABATT_CALL_ATTENTION || call == ABATT_CALL_FORWARD) {
@@ -211,31 +216,53 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     if (e != cudaSuccess) return ABATT_ERR_CUDA;
 
     __half *k16 = at<__half>(ws, L.k16);
-    e = launch_keys_f16(static_cast<const __nv_bfloat16 *>(K), k16, g.heads * g.N * g.d / 8, sms, st);
+    const bool coarse = cfg->scoring == ABATT_SCORE_BLOCK_MEANS;
+    // the scoring GEMM's key operand: fp16 keys, or fp16 block-mean keys
+    if (coarse)
+        e = launch_keys_block_mean(static_cast<const __nv_bfloat16 *>(K), k16, g.heads, g.N, g.d, g.Bk, g.nK,
+                                   sms, st);
+    else
+        e = launch_keys_f16(static_cast<const __nv_bfloat16 *>(K), k16, g.heads * g.N * g.d / 8, sms, st);
     if (e != cudaSuccess) return ABATT_ERR_CUDA;
 
     ScoreMaps sm;
     const int64_t MC = (int64_t)g.nQ * g.C;
+    const int nkeys = coarse ? g.nK : g.N;  // rows of the key operand per head
     if (!make_map(&sm.a, ka.cent16, g.d, MC, g.heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-        !make_map(&sm.k, k16, g.d, g.N, g.heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        !make_map(&sm.k, k16, g.d, nkeys, g.heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return ABATT_ERR_CUDA;
     ScoreArgs sa;
-    sa.heads = (int)g.heads; sa.N = g.N; sa.D = g.d; sa.Bk = g.Bk; sa.MC = (int)MC;
-    sa.nT = g.nT; sa.ldr = g.ldr;
-    score_chunks(g.nT, ((int)MC + 127) / 128 * g.heads, sms, &sa.nchunk, &sa.chunk_tiles);
+    sa.heads = (int)g.heads; sa.N = nkeys; sa.D = g.d; sa.Bk = coarse ? 1 : g.Bk; sa.MC = (int)MC;
+    sa.nT = coarse ? g.nTc : g.nT;
+    sa.ldr = coarse ? g.nTc * 128 : g.ldr;
+    // coarse: the last block's share is weighted by its valid keys over a full block
+    sa.last_weight = coarse ? (float)(g.N - (g.nK - 1) * g.Bk) / (float)g.Bk : 1.0f;
+    score_chunks(sa.nT, ((int)MC + 127) / 128 * g.heads, sms, &sa.nchunk, &sa.chunk_tiles);
     sa.r = at<float>(ws, L.r);
     sa.mref = at<float>(ws, L.mref);
     sa.mz = at<float2>(ws, L.mz);
     sa.hdr = at<WsHeader>(ws, L.hdr);
     sa.wait_ns = kWaitNs;
+    sa.C = g.C;
+    sa.weight = ka.weight;
+    sa.p = p;
+    sa.mode = 0;
+    if (coarse && 32 % g.C == 0) {
+        // two passes over the (cheap) block-mean GEMM: the centroids' softmax
+        // statistics, then p summed over each query block's centroid lanes
+        sa.mode = 1;
+        if ((e = launch_score(sa, sm, sms, st)) != cudaSuccess) return ABATT_ERR_CUDA;
+        sa.mode = 2;
+        return cuda_status(launch_score(sa, sm, sms, st));
+    }
     e = launch_score(sa, sm, sms, st);
     if (e != cudaSuccess) return ABATT_ERR_CUDA;
 
     CombineArgs ca;
-    ca.rows = g.rows; ca.C = g.C; ca.nK = g.nK; ca.nT = g.nT; ca.ldr = g.ldr; ca.Bk = g.Bk;
+    ca.rows = g.rows; ca.C = g.C; ca.nK = g.nK; ca.nT = sa.nT; ca.ldr = sa.ldr; ca.Bk = g.Bk;
     ca.r = sa.r; ca.mref = sa.mref; ca.weight = ka.weight; ca.mz = sa.mz; ca.p = p;
     ca.nchunk = sa.nchunk;
-    return cuda_status(launch_combine(ca, sms, st));
+    return cuda_status(coarse ? launch_combine_cols(ca, sms, st) : launch_combine(ca, sms, st));
 }
 
 abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, int32_t *counts,

@@ -31,7 +31,18 @@ struct ScoreArgs {
     int nT;        // key tiles per head, ceil(N/128)
     int ldr;       // row stride of r in floats (nT * 128/Bk)
     int nchunk;    // the key tiles are split into nchunk ranges of chunk_tiles (one CTA each)
+    float last_weight;  // coarse scoring (Bk == 1): weight of the last key column (n_last / Bk)
     int chunk_tiles;
+    // coarse scoring (Bk == 1) only:
+    //   mode 0: block values to r (+ mref), combined by launch_combine_cols;
+    //   mode 1: each centroid row's (max, sum) to mz only;
+    //   mode 2: p directly, from the merged (max, sum) of a mode-1 pass over the
+    //           same grid -- the C centroid rows of a query block are C adjacent
+    //           lanes of one warp, so C must divide 32
+    int mode;
+    int C;
+    const float *weight;  // [heads*MC] n_j / n (mode 2)
+    float *p;             // [heads*MC/C][N] (mode 2)
     float *r;      // [heads*MC][ldr]
     float *mref;   // [heads*MC][nT], running maximum within the tile's chunk
     float2 *mz;    // [heads*MC][nchunk] (max, sum) of each chunk in base 2
@@ -50,6 +61,11 @@ cudaError_t launch_score(const ScoreArgs &a, const ScoreMaps &maps, int num_sms,
 cudaError_t launch_keys_f16(const __nv_bfloat16 *K, __half *K16, int64_t n8, int num_sms,
                             cudaStream_t stream);
 
+// Mean key of every key block, to fp16 (coarse scoring): Kbar[head][b] =
+// mean of the block's valid keys.
+cudaError_t launch_keys_block_mean(const __nv_bfloat16 *K, __half *Kbar, int64_t heads, int N, int D,
+                                   int Bk, int nK, int num_sms, cudaStream_t stream);
+
 // Combine the C centroids of each query block into p (see score.cu).
 struct CombineArgs {
     int64_t rows;  // query blocks
@@ -59,6 +75,8 @@ struct CombineArgs {
     float *p;      // [rows][nK]
 };
 cudaError_t launch_combine(const CombineArgs &a, int num_sms, cudaStream_t stream);
+// Same for coarse scoring: r holds one value per key block, tiles of 128 blocks.
+cudaError_t launch_combine_cols(const CombineArgs &a, int num_sms, cudaStream_t stream);
 
 // ---- SIP sampler --------------------------------------------------------
 struct SampleArgs {

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             tc_fence_after();
             constexpr uint32_t idesc = idesc_f16(128, 128);
             const uint64_t da = sdesc_sw128(smem_u32(sA), 16, 1024);
+            const bool fill = BK != 1 || a.mode != 2;  // the epilogue leaves -m_ref in the buffer
             for (int i = 0; i < ntl; ++i) {
                 const int s = i % ST, buf = i % kScoreEpi, use = i / kScoreEpi;
                 if (!wait_all(&bar_kfull[s], (i / ST) & 1, 0x103)) break;
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
                     // after a buffer's first tile the epilogue leaves -m_ref in it:
                     // accumulate onto it, so the product arrives as x - m_ref
-                    umma_ss_w(d_tmem, da + off, kd + off, idesc, (kk > 0 || use > 0) ? 1u : 0u);
+                    umma_ss_w(d_tmem, da + off, kd + off, idesc, (kk > 0 || (use > 0 && fill)) ? 1u : 0u);
                 }
                 umma_commit_w(&bar_kempty[s]);
                 umma_commit_w(&bar_sfull[buf]);
@@ -191,6 +192,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const bool valid = grow < a.MC;
         const int64_t gr = (int64_t)hd * a.MC + grow;
         float m_run = kNegInf, Z = 0.0f;  // reference (base 2) and sum relative to it
+        // coarse mode 2: this row's final maximum m_j and log2(w_j / Z_j)
+        float mj = 0.0f, lfj = kNegInf;
+        if (BK == 1 && a.mode == 2 && valid) {
+            const float2 *q = a.mz + gr * a.nchunk;
+            float m = kNegInf;
+            for (int c = 0; c < a.nchunk; ++c) m = fmaxf(m, q[c].x);
+            float z = 0.0f;
+            for (int c = 0; c < a.nchunk; ++c)
+                if (q[c].x != kNegInf) z += q[c].y * ex2_approx(q[c].x - m);
+            const float w = a.weight[gr];
+            if (w > 0.0f && z > 0.0f) {
+                mj = m;
+                lfj = __log2f(w / z);
+            }
+        }
         for (int i = e; i < ntl; i += kScoreEpi) {
             const int kt = kt0 + i, use = i / kScoreEpi;
             if (!mbar_wait(&bar_sfull[e], use & 1, wc, 0x105)) break;
@@ -206,51 +222,63 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         if (q * 32 + c >= nvalid) v[c] = __float_as_uint(kNegInf);
                 }
             };
-            // block sums of 2^(y - sub) over the tile, y the buffer's values
-            constexpr int NA = BPT >= 8 ? 1 : 8 / BPT;
-            float bs[BPT];
-            auto block_sums = [&](float sub) {
-                const float2 nm = make_float2(-sub, -sub);
-                float2 acc[BPT][NA];
-#pragma unroll
-                for (int k = 0; k < BPT; ++k)
-#pragma unroll
-                    for (int u = 0; u < NA; ++u) acc[k][u] = make_float2(0.0f, 0.0f);
-#pragma unroll
+            bool emitted = false;
+            if constexpr (BK == 1) {
+              if (a.mode == 2) {
+                emitted = true;
+                // coarse scoring, second pass: e_{j,b} = (w_j/Z_j) 2^(x_jb - m_j), summed
+                // over the C centroid rows of each query block -- C adjacent lanes --
+                // by a butterfly reduce-scatter, after which lane g of a group holds
+                // the sums of W = 32/C consecutive columns and stores them to p
+                const int qi = grow / a.C;
+                float *prow = a.p + ((int64_t)hd * (a.MC / a.C) + qi) * a.N;
+                const int W = 32 / a.C;
+#pragma unroll 1
                 for (int q = 0; q < 4; ++q) {
                     uint32_t v[32];
                     load(q, v);
+                    const int col0 = kt * 128 + q * 32;
+                    float x[32];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const int col = q * 32 + c;
-                        float2 x = make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
-                        if (sub != 0.0f) x = __fadd2_rn(x, nm);
-                        float2 ex;
-                        if (((col >> 1) & 15) < kScorePolyOf16) {
-                            // the polynomial is valid below 2^128: larger inputs land at
-                            // 2^100 and send the tile to the exact path below
-                            x.x = fminf(x.x, 100.0f);
-                            x.y = fminf(x.y, 100.0f);
-                            ex = exp2_poly2<4>(x);
-                        } else {
-                            ex.x = ex2_approx(x.x);
-                            ex.y = ex2_approx(x.y);
+                    for (int c = 0; c < 32; ++c) x[c] = ex2_approx((__uint_as_float(v[c]) - mj) + lfj);
+                    const int lastc = a.N - 1 - col0;  // the last block, weighted by n_last / Bk
+                    if (lastc >= 0 && lastc < 32) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (c == lastc) x[c] *= a.last_weight;
+                    }
+                    int s = a.C >> 1;
+#pragma unroll
+                    for (int k = 0; k < 5; ++k) {
+                        const int half = 16 >> k;  // values exchanged at this step
+                        if (s > 0) {
+                            const bool hi = (lane & s) != 0;
+#pragma unroll
+                            for (int u = 0; u < half; ++u) {
+                                const float send = hi ? x[u] : x[u + half];
+                                const float keep = hi ? x[u + half] : x[u];
+                                x[u] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+                            }
+                            s >>= 1;
                         }
-                        float2 &s2 = acc[col / BK][(col >> 1) % NA];
-                        s2 = __fadd2_rn(s2, ex);
+                    }
+                    const int cb = col0 + (lane & (a.C - 1)) * W;
+                    if (valid) {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            if (k < W && cb + k < a.N) prow[cb + k] = x[k];
                     }
                 }
-#pragma unroll
-                for (int k = 0; k < BPT; ++k) {
-                    float2 t2 = acc[k][0];
-#pragma unroll
-                    for (int u = 1; u < NA; ++u) t2 = __fadd2_rn(t2, acc[k][u]);
-                    bs[k] = t2.x + t2.y;
-                }
-            };
-            // exact path: the tile's own maximum mx of y (relative to the current
-            // reference, or absolute on the first tile) becomes part of the reference
-            auto exact = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sempty[e]);
+              }
+            }
+            if (emitted) {
+            } else if constexpr (BK == 1) {
+                // coarse scoring: every column of the tile is one key block (its
+                // mean key); each tile takes the exact path and stores one value per
+                // column, the last block weighted by its share of a full block
                 float tq[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -270,37 +298,139 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 const float alpha = (m_run == kNegInf) ? 0.0f : ex2_approx(m_run - m_new);
                 Z *= alpha;
                 m_run = m_new;
-                block_sums(m_new - base);
-            };
-            // first tile of this buffer (the MMA started from zero): exact path;
-            // later tiles: the buffer held -m_run, so y = x - m_run already, one
-            // pass of exponentials -- unless some row's scores outgrew its
-            // reference, then the warp redoes the tile with the exact maximum
-            // (correct for every row; tensor-memory loads stay warp-uniform)
-            bool redo = use == 0;
-            if (!redo) {
-                block_sums(0.0f);
-                float big = 0.0f;
+                const float sub = m_new - base;
+                float zt = 0.0f;
 #pragma unroll
-                for (int k = 0; k < BPT; ++k) big = fmaxf(big, bs[k]);
-                redo = __any_sync(0xffffffffu, !(big < 0x1p80f));
-            }
-            if (redo) exact();
-            // leave -m_run in the buffer for its next tile, then free it
-            if (i + kScoreEpi < ntl) {
-                const uint32_t nmr = __float_as_uint(m_run == kNegInf ? 0.0f : -m_run);
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    load(q, v);
+                    float4 *dst = reinterpret_cast<float4 *>(a.r + gr * a.ldr + (int64_t)kt * 128 + q * 32);
+                    const int col0 = kt * 128 + q * 32;  // key column of v[0]
 #pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_fill32(taddr + q * 32, nmr);
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_sempty[e]);
+                    for (int c = 0; c < 32; c += 4) {
+                        float4 e4 = make_float4(ex2_approx(__uint_as_float(v[c]) - sub),
+                                                ex2_approx(__uint_as_float(v[c + 1]) - sub),
+                                                ex2_approx(__uint_as_float(v[c + 2]) - sub),
+                                                ex2_approx(__uint_as_float(v[c + 3]) - sub));
+                        const int last = a.N - 1 - (col0 + c);  // 0..3: the last block is here
+                        if (last >= 0 && last < 4) {
+                            if (last == 0) e4.x *= a.last_weight;
+                            else if (last == 1) e4.y *= a.last_weight;
+                            else if (last == 2) e4.z *= a.last_weight;
+                            else e4.w *= a.last_weight;
+                        }
+                        zt += (e4.x + e4.y) + (e4.z + e4.w);
+                        if (valid && a.mode == 0) dst[c / 4] = e4;
+                    }
+                }
+                Z += zt;
+                if (i + kScoreEpi < ntl) {
+                    const uint32_t nmr = __float_as_uint(m_run == kNegInf ? 0.0f : -m_run);
 #pragma unroll
-            for (int k = 0; k < BPT; ++k) Z += bs[k];
-            if (valid) {
-                store_blocks<BPT>(a.r + gr * a.ldr + (int64_t)kt * BPT, bs);
-                a.mref[gr * a.nT + kt] = m_run;
+                    for (int q = 0; q < 4; ++q) tmem_fill32(taddr + q * 32, nmr);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sempty[e]);
+                if (valid && a.mode == 0) a.mref[gr * a.nT + kt] = m_run;
+            } else {
+                // block sums of 2^(y - sub) over the tile, y the buffer's values
+                constexpr int NA = BPT >= 8 ? 1 : 8 / BPT;
+                float bs[BPT];
+                auto block_sums = [&](float sub) {
+                    const float2 nm = make_float2(-sub, -sub);
+                    float2 acc[BPT][NA];
+#pragma unroll
+                    for (int k = 0; k < BPT; ++k)
+#pragma unroll
+                        for (int u = 0; u < NA; ++u) acc[k][u] = make_float2(0.0f, 0.0f);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t v[32];
+                        load(q, v);
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const int col = q * 32 + c;
+                            float2 x = make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+                            if (sub != 0.0f) x = __fadd2_rn(x, nm);
+                            float2 ex;
+                            if (((col >> 1) & 15) < kScorePolyOf16) {
+                                // the polynomial is valid below 2^128: larger inputs land at
+                                // 2^100 and send the tile to the exact path below
+                                x.x = fminf(x.x, 100.0f);
+                                x.y = fminf(x.y, 100.0f);
+                                ex = exp2_poly2<4>(x);
+                            } else {
+                                ex.x = ex2_approx(x.x);
+                                ex.y = ex2_approx(x.y);
+                            }
+                            float2 &s2 = acc[col / BK][(col >> 1) % NA];
+                            s2 = __fadd2_rn(s2, ex);
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < BPT; ++k) {
+                        float2 t2 = acc[k][0];
+#pragma unroll
+                        for (int u = 1; u < NA; ++u) t2 = __fadd2_rn(t2, acc[k][u]);
+                        bs[k] = t2.x + t2.y;
+                    }
+                };
+                // exact path: the tile's own maximum mx of y (relative to the current
+                // reference, or absolute on the first tile) becomes part of the reference
+                auto exact = [&]() {
+                    float tq[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t v[32];
+                        load(q, v);
+                        float t0 = kNegInf, t1 = kNegInf;
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4) {
+                            t0 = fmax3f(t0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+                            t1 = fmax3f(t1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                        }
+                        tq[q] = fmaxf(t0, t1);
+                    }
+                    const float mx = fmaxf(fmax3f(tq[0], tq[1], tq[2]), tq[3]);
+                    const float base = (m_run == kNegInf) ? 0.0f : m_run;  // what y is relative to
+                    const float m_new = fmaxf(m_run, base + mx);
+                    const float alpha = (m_run == kNegInf) ? 0.0f : ex2_approx(m_run - m_new);
+                    Z *= alpha;
+                    m_run = m_new;
+                    block_sums(m_new - base);
+                };
+                // first tile of this buffer (the MMA started from zero): exact path;
+                // later tiles: the buffer held -m_run, so y = x - m_run already, one
+                // pass of exponentials -- unless some row's scores outgrew its
+                // reference, then the warp redoes the tile with the exact maximum
+                // (correct for every row; tensor-memory loads stay warp-uniform)
+                bool redo = use == 0;
+                if (!redo) {
+                    block_sums(0.0f);
+                    float big = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < BPT; ++k) big = fmaxf(big, bs[k]);
+                    redo = __any_sync(0xffffffffu, !(big < 0x1p80f));
+                }
+                if (redo) exact();
+                // leave -m_run in the buffer for its next tile, then free it
+                if (i + kScoreEpi < ntl) {
+                    const uint32_t nmr = __float_as_uint(m_run == kNegInf ? 0.0f : -m_run);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) tmem_fill32(taddr + q * 32, nmr);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_sempty[e]);
+#pragma unroll
+                for (int k = 0; k < BPT; ++k) Z += bs[k];
+                if (valid) {
+                    store_blocks<BPT>(a.r + gr * a.ldr + (int64_t)kt * BPT, bs);
+                    a.mref[gr * a.nT + kt] = m_run;
+                }
             }
         }
         mz_s[e][rl] = make_float2(m_run, Z);
@@ -317,7 +447,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 const float2 o = mz_s[g][rl];
                 if (o.x != kNegInf) z += o.y * ex2_approx(o.x - m);
             }
-            if (valid) a.mz[gr * a.nchunk + chunk] = make_float2(m, z);
+            if (valid && (BK != 1 || a.mode != 2)) a.mz[gr * a.nchunk + chunk] = make_float2(m, z);
         }
     }
     if (warp >= kWarpTma) {
@@ -420,6 +550,106 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     }
 }
 
+// ---- coarse scoring ------------------------------------------------------------
+// Kbar[h][b][x] = fp16 of the mean of K[h][b*Bk .. b*Bk + n_b)[x]; thread = (h, b, 8 dims)
+__global__ void __launch_bounds__(256) keys_block_mean_kernel(const __nv_bfloat16 *__restrict__ K,
+                                                              __half *__restrict__ Kbar, int64_t heads,
+                                                              int N, int D, int Bk, int nK) {
+    const int cpr = D / 8;  // 8-dim chunks per key
+    const int64_t total = heads * (int64_t)nK * cpr;
+    for (int64_t w = (int64_t)blockIdx.x * 256 + threadIdx.x; w < total; w += (int64_t)gridDim.x * 256) {
+        const int x8 = (int)(w % cpr);
+        const int64_t hb = w / cpr;
+        const int b = (int)(hb % nK);
+        const int64_t h = hb / nK;
+        const int n = min(Bk, N - b * Bk);
+        const uint4 *src = reinterpret_cast<const uint4 *>(K + ((h * N + (int64_t)b * Bk) * D)) + x8;
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int u = 0; u < n; ++u) {
+            const uint4 q = __ldg(src + (int64_t)u * cpr);
+            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                acc[2 * k] += __uint_as_float(wv[k] << 16);
+                acc[2 * k + 1] += __uint_as_float(wv[k] & 0xffff0000u);
+            }
+        }
+        const float inv = 1.0f / (float)n;
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float lo = fminf(fmaxf(acc[2 * k] * inv, -65504.0f), 65504.0f);
+            const float hi = fminf(fmaxf(acc[2 * k + 1] * inv, -65504.0f), 65504.0f);
+            const __half2 h2 = __floats2half2_rn(lo, hi);
+            o[k] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        reinterpret_cast<uint4 *>(Kbar + hb * D)[x8] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// p_b = sum_j (n_j/n) * r_{j,b} * 2^(mref_{j,b/128} - m_j) / Z_j, one thread per block
+__global__ void __launch_bounds__(256) combine_cols_kernel(const CombineArgs a) {
+    extern __shared__ float coef_s[];  // [C][nT]: (n_j/n) / Z_j * 2^(mref - m_j)
+    __shared__ float f_s[16], m_s[16];
+    for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
+        __syncthreads();
+        if (threadIdx.x < a.C) {
+            const int64_t j = row * a.C + threadIdx.x;
+            const float w = a.weight[j];
+            const float2 *mzj = a.mz + j * a.nchunk;
+            float m = kNegInf;
+            for (int c = 0; c < a.nchunk; ++c) m = fmaxf(m, mzj[c].x);
+            float z = 0.0f;
+            for (int c = 0; c < a.nchunk; ++c) {
+                const float2 q = mzj[c];
+                if (q.x != kNegInf) z += q.y * ex2_approx(q.x - m);
+            }
+            f_s[threadIdx.x] = (w > 0.0f && z > 0.0f) ? w / z : 0.0f;
+            m_s[threadIdx.x] = m;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < a.C * a.nT; e += blockDim.x) {
+            const int j = e / a.nT, T = e % a.nT;
+            const float f = f_s[j];
+            coef_s[e] = f == 0.0f ? 0.0f : f * ex2_approx(__ldg(a.mref + (row * a.C + j) * a.nT + T) - m_s[j]);
+        }
+        __syncthreads();
+        float *prow = a.p + row * (int64_t)a.nK;
+        // four blocks per thread (one float4 of r; rows of r are padded to 128
+        // columns, zeros past nK), the loads of four centroids in flight at once
+        for (int b = threadIdx.x * 4; b < a.nK; b += blockDim.x * 4) {
+            const int T = b >> 7;
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int j0 = 0; j0 < a.C; j0 += 4) {
+                float4 rv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    rv[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (j0 + u < a.C)
+                        rv[u] = __ldg(reinterpret_cast<const float4 *>(a.r + (row * a.C + j0 + u) * a.ldr + b));
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (j0 + u >= a.C) break;
+                    const float c = coef_s[(j0 + u) * a.nT + T];
+                    acc.x = fmaf(c, rv[u].x, acc.x);
+                    acc.y = fmaf(c, rv[u].y, acc.y);
+                    acc.z = fmaf(c, rv[u].z, acc.z);
+                    acc.w = fmaf(c, rv[u].w, acc.w);
+                }
+            }
+            if (b + 3 < a.nK && (a.nK & 3) == 0) {
+                *reinterpret_cast<float4 *>(prow + b) = acc;
+            } else {
+                const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (b + k < a.nK) prow[b + k] = v[k];
+            }
+        }
+    }
+}
+
 template <int D, int BK>
 cudaError_t launch_score_t(const ScoreArgs &a, const ScoreMaps &maps, cudaStream_t stream) {
     const size_t smem = (1 + kScoreStages) * (size_t)(128 * D * 2) + 1024;
@@ -434,6 +664,7 @@ cudaError_t launch_score_t(const ScoreArgs &a, const ScoreMaps &maps, cudaStream
 template <int D>
 cudaError_t launch_score_d(const ScoreArgs &a, const ScoreMaps &maps, cudaStream_t stream) {
     switch (a.Bk) {
+        case 1: return launch_score_t<D, 1>(a, maps, stream);  // coarse: one column per key block
         case 16: return launch_score_t<D, 16>(a, maps, stream);
         case 32: return launch_score_t<D, 32>(a, maps, stream);
         case 64: return launch_score_t<D, 64>(a, maps, stream);
@@ -457,6 +688,27 @@ cudaError_t launch_keys_f16(const __nv_bfloat16 *K, __half *K16, int64_t n8, int
     if (grid > cap) grid = cap;
     keys_f16_kernel<<<(unsigned)grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(K),
                                                         reinterpret_cast<uint4 *>(K16), n8);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_keys_block_mean(const __nv_bfloat16 *K, __half *Kbar, int64_t heads, int N, int D,
+                                   int Bk, int nK, int num_sms, cudaStream_t stream) {
+    const int64_t total = heads * (int64_t)nK * (D / 8);
+    if (total < 1) return cudaSuccess;
+    int64_t grid = (total + 255) / 256;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (grid > cap) grid = cap;
+    keys_block_mean_kernel<<<(unsigned)grid, 256, 0, stream>>>(K, Kbar, heads, N, D, Bk, nK);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_cols(const CombineArgs &a, int num_sms, cudaStream_t stream) {
+    int64_t grid = a.rows;
+    const int64_t cap = (int64_t)num_sms * 16;
+    if (grid > cap) grid = cap;
+    if (grid < 1) return cudaSuccess;
+    const size_t smem = sizeof(float) * (size_t)a.C * a.nT;
+    combine_cols_kernel<<<(unsigned)grid, 256, smem, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -76,6 +76,14 @@ typedef struct abatt_shape {
         (ABATT_ERR_UNSUPPORTED otherwise). */
 enum { ABATT_SELECT_SIP = 0, ABATT_SELECT_TOPK = 1 };
 
+/* How abatt_select scores the key blocks for a query block's centroids c_j.
+   KEYS: every key -- the block's share of centroid j's softmax over all keys.
+   BLOCK_MEANS: the coarse-summary baseline the abstract contrasts with -- each
+        block once, through the mean kbar_b of its keys, its share taken as
+        n_b * exp(scale * c_j . kbar_b) normalised over the blocks (n_b = valid
+        keys of b); Bk times less scoring work. */
+enum { ABATT_SCORE_KEYS = 0, ABATT_SCORE_BLOCK_MEANS = 1 };
+
 typedef struct abatt_config {
     int q_block;        /* Bq: queries per query block (128) */
     int kv_block;       /* Bk: keys per key/value block (16 by default) */
@@ -89,6 +97,7 @@ typedef struct abatt_config {
     int batch_offset;   /* global index of this call's first batch element (0 for a whole tensor) */
     int head_offset;    /* global index of this call's first head (0 for a whole tensor) */
     int selection;      /* ABATT_SELECT_SIP (0, the method) or ABATT_SELECT_TOPK (1) */
+    int scoring;        /* ABATT_SCORE_KEYS (0, the method as read) or ABATT_SCORE_BLOCK_MEANS (1) */
     /* The sampler's Philox counter uses the global indices (beta + batch_offset,
        h + head_offset), so a call over a slice of the batches or heads of a
        larger problem draws exactly the blocks that one call over the whole

@@ -293,8 +293,9 @@ def test_attention_empty_rows_and_bad_index():
 
 # --------------------------------------------------------------------------- selector
 
-def _select_check(Q, K, shape, C, I, Bk, rows_check=None):
-    cfg = abatt.Config(kv_block=Bk, clusters=C, kmeans_iters=I)
+def _select_check(Q, K, shape, C, I, Bk, rows_check=None, coarse=False):
+    cfg = abatt.Config(kv_block=Bk, clusters=C, kmeans_iters=I,
+                       scoring=abatt.SCORE_BLOCK_MEANS if coarse else abatt.SCORE_KEYS)
     p, cent, sizes = abatt.select(Q.cuda(), K.cuda(), cfg, want_centroids=True)
     p, cent, sizes = p.cpu().numpy(), cent.cpu().numpy(), sizes.cpu().numpy()
     rows = _rows_of(shape) if rows_check is None else np.asarray(rows_check)
@@ -303,7 +304,7 @@ def _select_check(Q, K, shape, C, I, Bk, rows_check=None):
     assert same_sizes.mean() >= 0.95
     ok = same_sizes
     assert np.max(np.abs(cent[rows][ok] - ocent[ok])) <= 1e-4 * max(1.0, np.abs(ocent).max())
-    p64, p32 = oracle.block_probs(Q, K, shape, rows, C, I, Bk=Bk)
+    p64, p32 = oracle.block_probs(Q, K, shape, rows, C, I, Bk=Bk, coarse=coarse)
     assert np.allclose(p.sum(1), 1.0, atol=2e-4)
     l1 = np.abs(p[rows][ok] - p64[ok]).sum(1)
     assert np.max(l1) <= 2e-3, np.max(l1)
@@ -337,6 +338,68 @@ def test_select_scores_that_grow_along_the_keys():
     Q = torch.from_numpy(q[None, None]).to(torch.bfloat16)
     K = torch.from_numpy(k[None, None]).to(torch.bfloat16)
     _select_check(Q, K, (1, 1, N, d), 2, 1, 16)
+
+
+# the coarse-summary scoring rule: each key block through its mean key
+
+def test_select_block_means_tiny():
+    w = synth.TINY
+    Q, K, V = synth.generate(w)
+    _select_check(Q, K, w.shape, w.clusters, w.iters, w.Bk, coarse=True)
+
+
+@pytest.mark.parametrize("N,Bk,C", [(1000, 16, 8), (1000, 64, 3), (1000, 128, 16), (5000, 16, 5),
+                                    (20000, 64, 16), (3000, 32, 1), (3000, 16, 2), (20000, 16, 4)])
+def test_select_block_means_ragged(N, Bk, C):
+    # partial last blocks (the n_b weight), several 128-block column tiles with a
+    # ragged last one, and (at 20000 keys) key ranges split over chunks; C that
+    # divides 32 takes the two-pass path that sums centroid lanes, C = 3 and 5
+    # the path through the block-value matrix
+    w = synth.WAN_1_3B.with_(H=2, N=N, grid=(1, 20, N // 20))
+    Q, K, V = synth.generate(w)
+    _select_check(Q, K, w.shape, C, 5, Bk, coarse=True)
+
+
+def test_select_block_means_d64_growing_keys():
+    # the keys of the per-key test above (their k-means has no near-ties)
+    N, d = 2048, 64
+    rng = np.random.default_rng(5)
+    u = rng.standard_normal(d)
+    g = np.linspace(1.0, 20.0, N)
+    q = np.tile(u, (N, 1)) + 0.05 * rng.standard_normal((N, d))
+    k = g[:, None] * u[None, :] + 0.05 * rng.standard_normal((N, d))
+    Q = torch.from_numpy(q[None, None]).to(torch.bfloat16)
+    K = torch.from_numpy(k[None, None]).to(torch.bfloat16)
+    _select_check(Q, K, (1, 1, N, d), 2, 1, 16, coarse=True)
+
+
+def test_forward_block_means_tiny():
+    # coarse scoring end to end: the sampler draws from the block-mean estimates
+    # exactly as the oracle does from the same probabilities, and attention runs
+    # on the drawn lists
+    w = synth.TINY
+    Q, K, V = synth.generate(w)
+    shape = w.shape
+    cfg = cfg_of(w, scoring=abatt.SCORE_BLOCK_MEANS)
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, shape, cfg), dtype=torch.uint8,
+                     device="cuda")
+    O = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg, workspace=ws)
+    torch.cuda.synchronize()
+    assert abatt.read_status(ws) == 0
+    p, counts, idx, logw = (t.cpu().numpy() for t in abatt.intermediates(ws, shape, cfg))
+    rows = _rows_of(shape)
+    p64, _ = oracle.block_probs(Q, K, shape, rows, w.clusters, w.iters, Bk=w.Bk, coarse=True)
+    assert np.max(np.abs(p[rows] - p64).sum(1)) <= 2e-3
+    oc, oi, ol, oamb, _ = oracle.sample(p, shape, rows, w.budget_bp, w.seed, Bk=w.Bk)
+    _check_lists_exact(counts, idx, logw, oc, oi, ol, oamb)
+    o5, _ = oracle.ht_attention(Q, K, V, shape, rows, counts, idx, logw, Bk=w.Bk)
+    Oc = O.float().cpu().numpy()
+    got = np.zeros_like(o5)
+    for r in rows:
+        h, q = divmod(int(r), w.nQ)
+        got[r] = Oc[0, h, q * 128:(q + 1) * 128]
+    assert _rel_l2(got, o5) <= REL_L2
+    assert np.max(np.abs(got - o5)) <= MAX_ABS
 
 
 # ------------------------------------------------------------------------- end to end
@@ -472,8 +535,9 @@ def test_forward_topk_tiny():
 
 
 def test_sip_and_topk_error_against_dense_attention(capsys):
-    # the comparison the abstract draws, on the same inputs and budget: SIP's
-    # reweighted draw against keeping the M largest estimates.  Reported
+    # the comparisons the abstract draws, on the same inputs and budget: SIP's
+    # reweighted draw against keeping the M largest estimates, each with per-key
+    # and with block-mean scoring.  Reported
     # (pytest -s), not judged: with V drawn as independent noise per token the
     # dense output is a small average over many keys, so every 10 % subset has
     # a large relative error here.  Asserted: keep-all reproduces dense
@@ -486,9 +550,13 @@ def test_sip_and_topk_error_against_dense_attention(capsys):
     rows = np.array([h * nQ + i for h in range(heads) for i in range(0, nQ, 16)])
     dense = oracle.dense_attention(Q, K, V, shape, rows)
     err = {}
-    for name, sel, bp in (("sip", abatt.SELECT_SIP, w.budget_bp), ("topk", abatt.SELECT_TOPK, w.budget_bp),
-                          ("keep-all", abatt.SELECT_SIP, 10000)):
-        cfg = cfg_of(w, selection=sel, budget_bp=bp)
+    means = abatt.SCORE_BLOCK_MEANS
+    for name, sel, bp, sc in (("sip", abatt.SELECT_SIP, w.budget_bp, 0),
+                              ("topk", abatt.SELECT_TOPK, w.budget_bp, 0),
+                              ("sip-means", abatt.SELECT_SIP, w.budget_bp, means),
+                              ("topk-means", abatt.SELECT_TOPK, w.budget_bp, means),
+                              ("keep-all", abatt.SELECT_SIP, 10000, 0)):
+        cfg = cfg_of(w, selection=sel, budget_bp=bp, scoring=sc)
         O = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg).float().cpu().numpy()
         got = np.stack([O[0, r // nQ, (r % nQ) * 128:(r % nQ + 1) * 128] for r in rows])
         n = [min(128, w.N - (r % nQ) * 128) for r in rows]
@@ -498,7 +566,8 @@ def test_sip_and_topk_error_against_dense_attention(capsys):
         err[name] = _rel_l2(got[mask], dense[mask])
     with capsys.disabled():
         print(f"\nrel L2 error vs dense attention at {w.budget_bp / 100:.0f} % budget "
-              f"({len(rows)} query blocks): SIP {err['sip']:.4f}, top-M {err['topk']:.4f}, "
+              f"({len(rows)} query blocks): SIP {err['sip']:.4f}, top-M {err['topk']:.4f}; "
+              f"block-mean scoring: SIP {err['sip-means']:.4f}, top-M {err['topk-means']:.4f}; "
               f"keep-all {err['keep-all']:.5f}")
     assert err["keep-all"] <= REL_L2
-    assert np.isfinite(err["sip"]) and np.isfinite(err["topk"])
+    assert all(np.isfinite(v) for v in err.values())
