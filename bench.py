@@ -53,18 +53,26 @@ def parse():
     return ap.parse_args()
 
 
+def attention_source(csrc: str) -> bytes:
+    """The source the gather-attention kernel is compiled from."""
+    head = open(os.path.join(csrc, "kernels.cuh"), "rb").read()
+    cut = head.find(b"// ---- gather attention")
+    return b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("attention.cu", "common.cuh")) + \
+        (head[cut:] if cut >= 0 else head)
+
+
 def attention_traffic(rows: int):
     """DRAM bytes of one gather_attn_kernel launch, from the committed ncu
     summary (bytes per query block, scaled by the launch's query blocks; DRAM
     traffic of the kernel is its compulsory Q/K/V/O bytes, which grow with the
     query blocks).  None when the kernel source differs from the one the
-    counters were taken on."""
+    counters were taken on: attention.cu, common.cuh and the gather-attention
+    part of kernels.cuh (from its "---- gather attention" heading on)."""
     import hashlib
     import re
     csrc = os.path.join(ROOT, "block_sparse_attention_20_b200", "csrc")
     try:
-        src = b"".join(open(os.path.join(csrc, f), "rb").read()
-                       for f in ("attention.cu", "common.cuh", "kernels.cuh"))
+        src = attention_source(csrc)
         txt = open(os.path.join(ROOT, "profiles", "gather_attn_kernel_wan1.3b.md")).read()
     except OSError:
         return None
