@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libabatt.so")
 CALL_SELECT, CALL_SAMPLE, CALL_ATTENTION, CALL_FORWARD = 0, 1, 2, 3
 SELECT_SIP, SELECT_TOPK = 0, 1
 SCORE_KEYS, SCORE_BLOCK_MEANS = 0, 1
+LAYOUT_BHND, LAYOUT_BNHD = 0, 1
 DEVFLAG_CAPACITY, DEVFLAG_TIMEOUT, DEVFLAG_BADLIST = 0x1, 0x2, 0x4
 
 # Every symbol declared in include/abatt.h.
@@ -47,7 +48,8 @@ class _Config(ctypes.Structure):
                 ("kmeans_iters", ctypes.c_int), ("budget_bp", ctypes.c_int),
                 ("scale", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("batch_offset", ctypes.c_int), ("head_offset", ctypes.c_int),
-                ("selection", ctypes.c_int), ("scoring", ctypes.c_int)]
+                ("selection", ctypes.c_int), ("scoring", ctypes.c_int),
+                ("layout", ctypes.c_int), ("reserved", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -65,12 +67,13 @@ class Config:
     head_offset: int = 0   # global index of the call's first head
     selection: int = 0     # SELECT_SIP (the method) or SELECT_TOPK (truncating baseline)
     scoring: int = 0       # SCORE_KEYS (the method as read) or SCORE_BLOCK_MEANS (coarse baseline)
+    layout: int = 0        # LAYOUT_BHND ([B,H,N,d]) or LAYOUT_BNHD ([B,N,H,d])
 
     def _c(self, d: int) -> _Config:
         s = self.scale if self.scale is not None else 1.0 / math.sqrt(d)
         return _Config(self.q_block, self.kv_block, self.clusters, self.kmeans_iters,
                        self.budget_bp, s, self.seed & (2**64 - 1), self.batch_offset, self.head_offset,
-                       self.selection, self.scoring)
+                       self.selection, self.scoring, self.layout, 0)
 
 
 _lock = threading.Lock()
@@ -134,8 +137,12 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _shape_of(q) -> _Shape:
-    B, H, N, d = q.shape
+def _shape_of(q, cfg=None) -> _Shape:
+    """(B, H, N, d) of a Q/K/V tensor in the layout cfg names."""
+    if cfg is not None and cfg.layout == LAYOUT_BNHD:
+        B, N, H, d = q.shape
+    else:
+        B, H, N, d = q.shape
     return _Shape(B, H, N, d)
 
 
@@ -149,7 +156,8 @@ def _check_bf16(*ts):
     import torch
     for t in ts:
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("Q, K, V must be contiguous CUDA bfloat16 tensors [B, H, N, d]")
+            raise ValueError("Q, K, V must be contiguous CUDA bfloat16 tensors ([B, H, N, d], or "
+                             "[B, N, H, d] with layout=LAYOUT_BNHD)")
 
 
 def workspace_size(call: int, shape, cfg: Config) -> int:
@@ -177,7 +185,7 @@ def select(q, k, cfg: Config, *, p=None, want_centroids=False, workspace=None, s
     cluster sizes [rows, C]."""
     import torch
     _check_bf16(q, k)
-    sh = _shape_of(q)
+    sh = _shape_of(q, cfg)
     nQ, nK, rows = _geom(sh, cfg)
     if p is None:
         p = torch.empty((rows, nK), dtype=torch.float32, device=q.device)
@@ -218,7 +226,7 @@ def attention(q, k, v, counts, idx, logw, cfg: Config, *, out=None, want_lse=Fal
     """Gather attention over the listed blocks.  Returns O (and lse)."""
     import torch
     _check_bf16(q, k, v)
-    sh = _shape_of(q)
+    sh = _shape_of(q, cfg)
     cap = idx.shape[1]
     if out is None:
         out = torch.empty_like(q)
@@ -243,7 +251,7 @@ def attention_noalloc(q, k, v, counts, idx, logw, cfg: Config, *, out, lse=None,
     that overlap on the GPU race on it).  The caller supplies every input and
     output buffer, including `out` (and `lse`, `dev_status` if wanted)."""
     _check_bf16(q, k, v)
-    sh = _shape_of(q)
+    sh = _shape_of(q, cfg)
     _check(lib().abatt_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(sh),
                                          ctypes.byref(cfg._c(sh.d)), _ptr(counts), _ptr(idx),
                                          _ptr(logw), idx.shape[1], _ptr(out), _ptr(lse),
@@ -257,7 +265,7 @@ def forward(q, k, v, cfg: Config, *, out=None, want_lse=False, workspace=None, s
     intermediates (see :func:`intermediates`)."""
     import torch
     _check_bf16(q, k, v)
-    sh = _shape_of(q)
+    sh = _shape_of(q, cfg)
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((sh.B, sh.H, sh.N), dtype=torch.float32, device=q.device) if want_lse else None
@@ -283,6 +291,8 @@ class HostPipeline:
 
     def __init__(self, shape, cfg: Config, *, heads_per_chunk: int = 5, device=None):
         import torch
+        if cfg.layout != LAYOUT_BHND:
+            raise ValueError("HostPipeline streams head chunks of [B, H, N, d] tensors (layout=LAYOUT_BHND)")
         self.B, self.H, self.N, self.d = shape
         self.cfg = cfg
         self.hc = max(1, min(heads_per_chunk, self.H))

@@ -24,6 +24,20 @@ struct Geom {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+Strides strides_of(const Geom &g, const abatt_config *cfg) {
+    Strides s;
+    s.H = g.H;
+    if (cfg->layout == ABATT_LAYOUT_BNHD) {
+        s.sT = (int64_t)g.H * g.d;
+        s.sH = g.d;
+    } else {
+        s.sT = g.d;
+        s.sH = (int64_t)g.N * g.d;
+    }
+    s.sB = (int64_t)g.H * g.N * g.d;
+    return s;
+}
+
 // The scoring kernel runs one CTA per (centroid tile, head, key-range chunk),
 // one CTA per SM at a time.  Split the key tiles into the fewest chunks (at
 // most kMaxScoreChunks, each of at least 24 tiles) whose CTA count fills its
@@ -55,6 +69,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (c->batch_offset < 0 || c->head_offset < 0) return ABATT_ERR_INVALID_ARG;
     if (c->selection != ABATT_SELECT_SIP && c->selection != ABATT_SELECT_TOPK) return ABATT_ERR_INVALID_ARG;
     if (c->scoring != ABATT_SCORE_KEYS && c->scoring != ABATT_SCORE_BLOCK_MEANS) return ABATT_ERR_INVALID_ARG;
+    if (c->layout != ABATT_LAYOUT_BHND && c->layout != ABATT_LAYOUT_BNHD) return ABATT_ERR_INVALID_ARG;
     if (s->d != 64 && s->d != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->q_block != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->kv_block != 16 && c->kv_block != 32 && c->kv_block != 64 && c->kv_block != 128)
@@ -173,14 +188,15 @@ bool make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int64_t out
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 4-D bf16 map with 128-byte swizzle and a 64-element inner box.
-bool make_map4(CUtensorMap *m, const void *base, const cuuint64_t dims[4],
-               const cuuint64_t strides[3], const cuuint32_t box[4]) {
+// bf16 map of `rank` dimensions (dims[0] innermost, strides in bytes of
+// dims 1..rank-1) with 128-byte swizzle and a 64-element inner box.
+bool make_map_nd(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                 const cuuint64_t *strides, const cuuint32_t *box) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -206,6 +222,7 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
                         int sms, cudaStream_t st) {
     KmeansArgs ka;
     ka.Q = static_cast<const __nv_bfloat16 *>(Q);
+    ka.st = strides_of(g, cfg);
     ka.rows = g.rows; ka.nQ = g.nQ; ka.N = g.N; ka.D = g.d; ka.C = g.C; ka.iters = g.I;
     ka.logit_mul = cfg->scale * kLog2eF;
     ka.cent16 = at<__half>(ws, L.cent16);
@@ -218,11 +235,13 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     __half *k16 = at<__half>(ws, L.k16);
     const bool coarse = cfg->scoring == ABATT_SCORE_BLOCK_MEANS;
     // the scoring GEMM's key operand: fp16 keys, or fp16 block-mean keys
+    const __nv_bfloat16 *Kb = static_cast<const __nv_bfloat16 *>(K);
     if (coarse)
-        e = launch_keys_block_mean(static_cast<const __nv_bfloat16 *>(K), k16, g.heads, g.N, g.d, g.Bk, g.nK,
-                                   sms, st);
+        e = launch_keys_block_mean(Kb, ka.st, k16, g.heads, g.N, g.d, g.Bk, g.nK, sms, st);
+    else if (cfg->layout == ABATT_LAYOUT_BHND)
+        e = launch_keys_f16(Kb, k16, g.heads * g.N * g.d / 8, sms, st);
     else
-        e = launch_keys_f16(static_cast<const __nv_bfloat16 *>(K), k16, g.heads * g.N * g.d / 8, sms, st);
+        e = launch_keys_f16_strided(Kb, ka.st, k16, g.heads, g.N, g.d, sms, st);
     if (e != cudaSuccess) return ABATT_ERR_CUDA;
 
     ScoreMaps sm;
@@ -296,26 +315,44 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     if (launch_pair_union(pa, sms, st) != cudaSuccess) return ABATT_ERR_CUDA;
 
     const int CH = g.d / 64;
-    const bool fold = (g.N % 8) == 0 && g.heads * (g.N / 8) < (int64_t(1) << 31);
+    const Strides sd = strides_of(g, cfg);
+    const bool bnhd = cfg->layout == ABATT_LAYOUT_BNHD;
+    // K as boxes of 8-row groups: the batch index folds into the group index
+    // ([B][N][H][d]: sB = N*sT) or into the outer index ([B][H][N][d]: sB = H*sH)
+    const int64_t groups = bnhd ? (int64_t)g.B * (g.N / 8) : g.N / 8;
+    const int64_t outer = bnhd ? g.H : g.heads;
+    const bool fold = (g.N % 8) == 0 && groups < (int64_t(1) << 31) && outer < (int64_t(1) << 31);
+    const cuuint64_t sT2 = (cuuint64_t)sd.sT * 2, sH2 = (cuuint64_t)sd.sH * 2, sB2 = (cuuint64_t)sd.sB * 2;
     AttnMaps m;
-    if (!make_map(&m.q, Q, g.d, g.N, g.heads, 128)) return ABATT_ERR_CUDA;
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.H, (cuuint64_t)g.B};
+        const cuuint64_t strides[3] = {sT2, sH2, sB2};
+        const cuuint32_t box[4] = {64, 128, 1, 1};
+        if (!make_map_nd(&m.q, Q, 4, dims, strides, box)) return ABATT_ERR_CUDA;
+    }
     if (fold) {
-        const cuuint64_t dims[4] = {64, 8, (cuuint64_t)CH, (cuuint64_t)(g.heads * (g.N / 8))};
-        const cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, 128, (cuuint64_t)8 * g.d * 2};
-        const cuuint32_t box[4] = {64, 8, (cuuint32_t)CH, (cuuint32_t)(g.Bk / 8)};
-        if (!make_map4(&m.k, K, dims, strides, box)) return ABATT_ERR_CUDA;
-    } else if (!make_map(&m.k, K, g.d, g.N, g.heads, g.Bk)) {
-        return ABATT_ERR_CUDA;
+        const cuuint64_t dims[5] = {64, 8, (cuuint64_t)CH, (cuuint64_t)groups, (cuuint64_t)outer};
+        const cuuint64_t strides[4] = {sT2, 128, 8 * sT2, sH2};
+        const cuuint32_t box[5] = {64, 8, (cuuint32_t)CH, (cuuint32_t)(g.Bk / 8), 1};
+        if (!make_map_nd(&m.k, K, 5, dims, strides, box)) return ABATT_ERR_CUDA;
+    } else {
+        const cuuint64_t dims[4] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.H, (cuuint64_t)g.B};
+        const cuuint64_t strides[3] = {sT2, sH2, sB2};
+        const cuuint32_t box[4] = {64, (cuuint32_t)g.Bk, 1, 1};
+        if (!make_map_nd(&m.k, K, 4, dims, strides, box)) return ABATT_ERR_CUDA;
     }
     {
-        const cuuint64_t dims[4] = {64, (cuuint64_t)g.N, (cuuint64_t)CH, (cuuint64_t)g.heads};
-        const cuuint64_t strides[3] = {(cuuint64_t)g.d * 2, 128, (cuuint64_t)g.N * g.d * 2};
-        const cuuint32_t box[4] = {64, (cuuint32_t)g.Bk, (cuuint32_t)CH, 1};
-        if (!make_map4(&m.v, V, dims, strides, box)) return ABATT_ERR_CUDA;
+        const cuuint64_t dims[5] = {64, (cuuint64_t)g.N, (cuuint64_t)CH, (cuuint64_t)g.H, (cuuint64_t)g.B};
+        const cuuint64_t strides[4] = {sT2, 128, sH2, sB2};
+        const cuuint32_t box[5] = {64, (cuuint32_t)g.Bk, (cuuint32_t)CH, 1, 1};
+        if (!make_map_nd(&m.v, V, 5, dims, strides, box)) return ABATT_ERR_CUDA;
     }
     AttnArgs a;
     a.rows = g.rows; a.pairs = pairs_of(g); a.nQ = g.nQ; a.N = g.N; a.D = g.d; a.Bk = g.Bk;
     a.nK = g.nK; a.cap_u = g.nK; a.k_fold = fold ? 1 : 0;
+    a.kf_gb = bnhd ? g.N / 8 : 0;
+    a.kf_zb = bnhd ? 0 : g.H;
+    a.st = sd;
     a.scale_log2 = cfg->scale * kLog2eF;
     a.useg = pa.useg; a.ublk = pa.ublk; a.ulw = pa.ulw;
     a.O = static_cast<__nv_bfloat16 *>(O);

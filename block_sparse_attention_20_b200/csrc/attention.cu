@@ -291,7 +291,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_prefetch_desc(&maps.k);
             tma_prefetch_desc(&maps.v);
         }
-        const int groups_per_head = a.N / 8;
         uint32_t q_loads[2] = {0, 0};
         uint32_t rp = 0;
         bool ok = true;
@@ -301,6 +300,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const PairPlan P(a.useg, pr, rr[1] >= 0, BPT);
             if (P.groups == 0) continue;
             const int hd = (int)(rr[0] / a.nQ);
+            const int bat = hd / a.st.H, hed = hd % a.st.H;  // batch element and head
             const int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
             // block index of this lane in gather group g (-1: empty slot)
             auto blk_of = [&](int g) -> int {
@@ -320,9 +320,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&bar_qf[s], TILE);
-                    const int i = (int)(row % a.nQ), h = (int)(row / a.nQ);
+                    const int i = (int)(row % a.nQ);
                     for (int c = 0; c < CH; ++c)
-                        tma_load_3d(sQ + s * TILE + c * 16384, &maps.q, &bar_qf[s], c * 64, i * 128, h);
+                        tma_load_4d(sQ + s * TILE + c * 16384, &maps.q, &bar_qf[s], c * 64, i * 128, hed, bat);
                     ++q_loads[s];
                 }
             }
@@ -343,18 +343,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const bool valid = blk >= 0;
                         if (kv == 0) {
                             if (KFOLD) {
-                                // groups of 8 rows with all heads folded: a box of Bk/8 groups
-                                const int gi = valid ? hd * groups_per_head + blk * (BK / 8) : 0x7fffff00;
-                                tma_load_4d(dst + lane * BLK, &maps.k, &bar_kvf[stg], 0, 0, 0, gi);
+                                // a box of Bk/8 groups of 8 rows, all head-dim chunks
+                                const int gy = valid ? bat * a.kf_gb + blk * (BK / 8) : 0x7fffff00;
+                                tma_load_5d(dst + lane * BLK, &maps.k, &bar_kvf[stg], 0, 0, 0, gy,
+                                            bat * a.kf_zb + hed);
                             } else {
                                 const int y = valid ? blk * BK : a.nK * BK;
                                 for (int c = 0; c < CH; ++c)
-                                    tma_load_3d(dst + c * 16384 + lane * BK * 128, &maps.k, &bar_kvf[stg],
-                                                c * 64, y, hd);
+                                    tma_load_4d(dst + c * 16384 + lane * BK * 128, &maps.k, &bar_kvf[stg],
+                                                c * 64, y, hed, bat);
                             }
                         } else {
                             const int y = valid ? blk * BK : a.nK * BK;
-                            tma_load_4d(dst + lane * BLK, &maps.v, &bar_kvf[stg], 0, y, 0, hd);
+                            tma_load_5d(dst + lane * BLK, &maps.v, &bar_kvf[stg], 0, y, 0, hed, bat);
                         }
                     }
                     ++rp;
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 m_run = m_use;
             }
             if (!ok) break;
-            __nv_bfloat16 *orow = a.O + tok * D + hh * (D / 2);
+            __nv_bfloat16 *orow = a.O + a.st.head_base(hd) + (int64_t)(i * 128 + r) * a.st.sT + hh * (D / 2);
             if (n == 0) {  // no block at all: O = 0, lse = -inf
                 if (r < nrows) {
 #pragma unroll

@@ -5,9 +5,19 @@
 
 namespace abatt {
 
+// Element strides of Q, K, V, O: element (beta, h, t, x) sits at
+// beta*sB + h*sH + t*sT + x.  [B][H][N][d]: sT = d, sH = N*d, sB = H*N*d;
+// [B][N][H][d]: sT = H*d, sH = d, sB = N*H*d.
+struct Strides {
+    int64_t sT, sH, sB;
+    int H;
+    __host__ __device__ int64_t head_base(int64_t bh) const { return (bh / H) * sB + (bh % H) * sH; }
+};
+
 // ---- IBCS part 1: per-query-block k-means ---------------------------------
 struct KmeansArgs {
-    const __nv_bfloat16 *Q;  // [B*H][N][D]
+    const __nv_bfloat16 *Q;  // strided as st
+    Strides st;
     int64_t rows;            // B*H*nQ
     int nQ, N, D, C, iters;
     float logit_mul;         // scale * log2(e), folded into the GEMM operand
@@ -60,11 +70,14 @@ cudaError_t launch_score(const ScoreArgs &a, const ScoreMaps &maps, int num_sms,
 // normal range; magnitudes beyond 65504 saturate).  n8 = elements / 8.
 cudaError_t launch_keys_f16(const __nv_bfloat16 *K, __half *K16, int64_t n8, int num_sms,
                             cudaStream_t stream);
+// Same from strided keys: K16[bh][t] = K at (bh, t), heads*N rows of D.
+cudaError_t launch_keys_f16_strided(const __nv_bfloat16 *K, const Strides &st, __half *K16, int64_t heads,
+                                    int N, int D, int num_sms, cudaStream_t stream);
 
 // Mean key of every key block, to fp16 (coarse scoring): Kbar[head][b] =
 // mean of the block's valid keys.
-cudaError_t launch_keys_block_mean(const __nv_bfloat16 *K, __half *Kbar, int64_t heads, int N, int D,
-                                   int Bk, int nK, int num_sms, cudaStream_t stream);
+cudaError_t launch_keys_block_mean(const __nv_bfloat16 *K, const Strides &st, __half *Kbar, int64_t heads,
+                                   int N, int D, int Bk, int nK, int num_sms, cudaStream_t stream);
 
 // Combine the C centroids of each query block into p (see score.cu).
 struct CombineArgs {
@@ -130,20 +143,22 @@ struct AttnArgs {
     int64_t rows, pairs;  // query blocks, row pairs
     int nQ, N, D, Bk, nK;
     int cap_u;
-    int k_fold;        // K tiles via head-folded 4-D boxes (needs N % 8 == 0)
+    int k_fold;        // K tiles as boxes of 8-row groups (needs N % 8 == 0)
+    int kf_gb, kf_zb;  // k_fold: group coordinate b*kf_gb + blk*Bk/8, outer coordinate b*kf_zb + h
+    Strides st;        // of O (and of Q, K, V in the maps)
     float scale_log2;  // scale * log2(e)
     const int32_t *useg, *ublk;
     const float *ulw;
-    __nv_bfloat16 *O;  // [B*H][N][D]
+    __nv_bfloat16 *O;  // strided as st
     float *lse;        // optional [B*H][N]
     WsHeader *hdr;
     uint64_t wait_ns;
 };
 struct AttnMaps {
-    CUtensorMap q;  // [heads][N][D], box (64, 128, 1)
-    CUtensorMap k;  // k_fold: (64, 8 rows, 2 chunks, heads*N/8 groups), box (64, 8, 2, Bk/8)
-                    // else:   [heads][N][D], box (64, Bk, 1)
-    CUtensorMap v;  // (64, N rows, 2 chunks, heads), box (64, Bk, 2, 1)
+    CUtensorMap q;  // (D, N, H, B), box (64, 128, 1, 1)
+    CUtensorMap k;  // k_fold: (64, 8 rows, D/64 chunks, groups, outer), box (64, 8, D/64, Bk/8, 1)
+                    // else:   (D, N, H, B), box (64, Bk, 1, 1)
+    CUtensorMap v;  // (64, N rows, D/64 chunks, H, B), box (64, Bk, D/64, 1, 1)
 };
 cudaError_t launch_attention(const AttnArgs &a, const AttnMaps &maps, int num_sms,
                              cudaStream_t stream);

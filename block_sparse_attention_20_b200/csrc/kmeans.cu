@@ -83,18 +83,18 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         const int64_t bh = row / a.nQ;
         const int n = min(128, a.N - i * 128);
         const int ce = min(C, n);
-        const __nv_bfloat16 *qblk = a.Q + (bh * (int64_t)a.N + (int64_t)i * 128) * D;
+        const __nv_bfloat16 *qblk = a.Q + a.st.head_base(bh) + (int64_t)i * 128 * a.st.sT;
 
-        // the block's queries (contiguous in memory: coalesced 16-byte chunks);
-        // missing rows are zero
+        // the block's queries (each row's 16-byte chunks coalesced; rows sT
+        // apart); missing rows are zero
         {
             constexpr int CPR = D / 8;  // 16-byte chunks per row
-            const uint4 *src = reinterpret_cast<const uint4 *>(qblk);
 #pragma unroll 4
             for (int c = tid; c < 128 * CPR; c += kKmThreads) {
                 const int r = c / CPR, x8 = c % CPR;
                 *reinterpret_cast<uint4 *>(qs + r * LDQ + x8 * 8) =
-                    r < n ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+                    r < n ? __ldg(reinterpret_cast<const uint4 *>(qblk + (int64_t)r * a.st.sT) + x8)
+                          : make_uint4(0, 0, 0, 0);
             }
         }
         __syncthreads();

@@ -61,6 +61,22 @@ __global__ void __launch_bounds__(256) keys_f16_kernel(const uint4 *__restrict__
     }
 }
 
+// strided keys: thread = (row bh*N + t, 8 dims)
+__global__ void __launch_bounds__(256) keys_f16_strided_kernel(const __nv_bfloat16 *__restrict__ K,
+                                                               const Strides st, uint4 *__restrict__ dst,
+                                                               int64_t heads, int N, int D) {
+    const int cpr = D / 8;
+    const int64_t total = heads * (int64_t)N * cpr;
+    for (int64_t w = (int64_t)blockIdx.x * 256 + threadIdx.x; w < total; w += (int64_t)gridDim.x * 256) {
+        const int x8 = (int)(w % cpr);
+        const int64_t row = w / cpr;
+        const int t = (int)(row % N);
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(K + st.head_base(row / N) + t * st.sT) + x8);
+        dst[w] = make_uint4(bf16x2_to_f16x2_sat(u.x), bf16x2_to_f16x2_sat(u.y), bf16x2_to_f16x2_sat(u.z),
+                            bf16x2_to_f16x2_sat(u.w));
+    }
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -553,8 +569,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 // ---- coarse scoring ------------------------------------------------------------
 // Kbar[h][b][x] = fp16 of the mean of K[h][b*Bk .. b*Bk + n_b)[x]; thread = (h, b, 8 dims)
 __global__ void __launch_bounds__(256) keys_block_mean_kernel(const __nv_bfloat16 *__restrict__ K,
-                                                              __half *__restrict__ Kbar, int64_t heads,
-                                                              int N, int D, int Bk, int nK) {
+                                                              const Strides st, __half *__restrict__ Kbar,
+                                                              int64_t heads, int N, int D, int Bk, int nK) {
     const int cpr = D / 8;  // 8-dim chunks per key
     const int64_t total = heads * (int64_t)nK * cpr;
     for (int64_t w = (int64_t)blockIdx.x * 256 + threadIdx.x; w < total; w += (int64_t)gridDim.x * 256) {
@@ -563,10 +579,10 @@ __global__ void __launch_bounds__(256) keys_block_mean_kernel(const __nv_bfloat1
         const int b = (int)(hb % nK);
         const int64_t h = hb / nK;
         const int n = min(Bk, N - b * Bk);
-        const uint4 *src = reinterpret_cast<const uint4 *>(K + ((h * N + (int64_t)b * Bk) * D)) + x8;
+        const __nv_bfloat16 *src = K + st.head_base(h) + (int64_t)b * Bk * st.sT + x8 * 8;
         float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         for (int u = 0; u < n; ++u) {
-            const uint4 q = __ldg(src + (int64_t)u * cpr);
+            const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)u * st.sT));
             const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -691,14 +707,26 @@ cudaError_t launch_keys_f16(const __nv_bfloat16 *K, __half *K16, int64_t n8, int
     return cudaGetLastError();
 }
 
-cudaError_t launch_keys_block_mean(const __nv_bfloat16 *K, __half *Kbar, int64_t heads, int N, int D,
-                                   int Bk, int nK, int num_sms, cudaStream_t stream) {
+cudaError_t launch_keys_f16_strided(const __nv_bfloat16 *K, const Strides &st, __half *K16, int64_t heads,
+                                    int N, int D, int num_sms, cudaStream_t stream) {
+    const int64_t total = heads * (int64_t)N * (D / 8);
+    if (total < 1) return cudaSuccess;
+    int64_t grid = (total + 255) / 256;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (grid > cap) grid = cap;
+    keys_f16_strided_kernel<<<(unsigned)grid, 256, 0, stream>>>(K, st, reinterpret_cast<uint4 *>(K16), heads,
+                                                                N, D);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_keys_block_mean(const __nv_bfloat16 *K, const Strides &st, __half *Kbar, int64_t heads,
+                                   int N, int D, int Bk, int nK, int num_sms, cudaStream_t stream) {
     const int64_t total = heads * (int64_t)nK * (D / 8);
     if (total < 1) return cudaSuccess;
     int64_t grid = (total + 255) / 256;
     const int64_t cap = (int64_t)num_sms * 8;
     if (grid > cap) grid = cap;
-    keys_block_mean_kernel<<<(unsigned)grid, 256, 0, stream>>>(K, Kbar, heads, N, D, Bk, nK);
+    keys_block_mean_kernel<<<(unsigned)grid, 256, 0, stream>>>(K, st, Kbar, heads, N, D, Bk, nK);
     return cudaGetLastError();
 }
 

@@ -17,7 +17,9 @@
  *     The caller owns every buffer; the library never allocates or frees
  *     memory and keeps no state between calls other than cached kernel
  *     attributes.
- *   - Q, K, V, O: bf16, contiguous [B][H][N][d], 16-byte aligned base.
+ *   - Q, K, V, O: bf16, 16-byte aligned base, contiguous in the layout
+ *     cfg->layout names: [B][H][N][d] (ABATT_LAYOUT_BHND, the default) or
+ *     [B][N][H][d] (ABATT_LAYOUT_BNHD).  lse is [B][H][N] in both.
  *   - A "row" is one query block (beta, h, i), linear id
  *     ((beta*H)+h)*nQ + i, with nQ = ceil(N/q_block), nK = ceil(N/kv_block).
  *     The last query block and the last key block may be partial; missing
@@ -76,6 +78,14 @@ typedef struct abatt_shape {
         (ABATT_ERR_UNSUPPORTED otherwise). */
 enum { ABATT_SELECT_SIP = 0, ABATT_SELECT_TOPK = 1 };
 
+/* Memory layout of Q, K, V and O.
+   BHND: [B][H][N][d] -- each head's tokens contiguous.
+   BNHD: [B][N][H][d] -- token-major with the heads interleaved, as the
+        query/key/value projections of a transformer block emit them and its
+        output projection reads them, so no transpose is needed around a call.
+   Results are bit-identical between the two layouts. */
+enum { ABATT_LAYOUT_BHND = 0, ABATT_LAYOUT_BNHD = 1 };
+
 /* How abatt_select scores the key blocks for a query block's centroids c_j.
    KEYS: every key -- the block's share of centroid j's softmax over all keys.
    BLOCK_MEANS: the coarse-summary baseline the abstract contrasts with -- each
@@ -98,6 +108,8 @@ typedef struct abatt_config {
     int head_offset;    /* global index of this call's first head (0 for a whole tensor) */
     int selection;      /* ABATT_SELECT_SIP (0, the method) or ABATT_SELECT_TOPK (1) */
     int scoring;        /* ABATT_SCORE_KEYS (0, the method as read) or ABATT_SCORE_BLOCK_MEANS (1) */
+    int layout;         /* ABATT_LAYOUT_BHND (0) or ABATT_LAYOUT_BNHD (1) */
+    int reserved;       /* set to 0 */
     /* The sampler's Philox counter uses the global indices (beta + batch_offset,
        h + head_offset), so a call over a slice of the batches or heads of a
        larger problem draws exactly the blocks that one call over the whole

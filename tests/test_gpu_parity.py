@@ -402,6 +402,55 @@ def test_forward_block_means_tiny():
     assert np.max(np.abs(got - o5)) <= MAX_ABS
 
 
+# ------------------------------------------------------------------- [B, N, H, d] layout
+
+def _forward_all(Q, K, V, shape, cfg):
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, shape, cfg), dtype=torch.uint8,
+                     device="cuda")
+    O, lse = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg, workspace=ws, want_lse=True)
+    torch.cuda.synchronize()
+    assert abatt.read_status(ws) == 0
+    return O.cpu(), lse.cpu(), [t.cpu() for t in abatt.intermediates(ws, shape, cfg)]
+
+
+@pytest.mark.parametrize("B,H,N,d,Bk,scoring", [
+    (2, 3, 1000, 64, 16, 0),    # key groups of 8 rows (N % 8 == 0), ragged last query block, two batches
+    (1, 2, 1001, 128, 32, 0),   # per-block key boxes (N % 8 != 0)
+    (2, 2, 4096, 128, 64, 0),
+    (1, 3, 777, 64, 128, 0),
+    (2, 2, 1000, 128, 16, 1),   # block-mean scoring over strided keys
+])
+def test_layout_bnhd_is_bit_identical(B, H, N, d, Bk, scoring):
+    # the same problem stored token-major ([B, N, H, d]) gives the same bits:
+    # the same queries enter k-means, the same keys the scoring GEMM, the same
+    # rows the attention tiles -- only the addresses differ
+    w = synth.WAN_1_3B.with_(B=B, H=H, N=N, d=d, grid=(1, 10, -(-N // 10)))
+    Q, K, V = synth.generate(w)
+    shape = (B, H, N, d)
+    cfg = abatt.Config(kv_block=Bk, clusters=8, kmeans_iters=5, budget_bp=1500, seed=99, scoring=scoring)
+    O1, lse1, mid1 = _forward_all(Q, K, V, shape, cfg)
+    t = lambda x: x.permute(0, 2, 1, 3).contiguous()
+    cfg2 = abatt.Config(**{**cfg.__dict__, "layout": abatt.LAYOUT_BNHD})
+    O2, lse2, mid2 = _forward_all(t(Q), t(K), t(V), shape, cfg2)
+    assert O2.shape == (B, N, H, d)
+    for a_, b_ in zip(mid1, mid2):
+        assert torch.equal(a_, b_)
+    assert torch.equal(lse1, lse2)
+    assert torch.equal(O1, O2.permute(0, 2, 1, 3))
+    # and it is attention: the kernel's output against the oracle on its lists
+    p, counts, idx, logw = (x.numpy() for x in mid1)
+    rows = np.arange(0, len(counts), max(1, len(counts) // 24))
+    o5, _ = oracle.ht_attention(Q, K, V, shape, rows, counts[rows], idx[rows], logw[rows], Bk=Bk)
+    nQ = -(-N // 128)
+    got = np.zeros_like(o5)
+    Of = O1.float().numpy()
+    for k, r in enumerate(rows):
+        bh, q = divmod(int(r), nQ)
+        n = min(128, N - q * 128)
+        got[k, :n] = Of[bh // H, bh % H, q * 128:q * 128 + n]
+    assert _rel_l2(got, o5) <= REL_L2
+
+
 # ------------------------------------------------------------------------- end to end
 
 def _forward_check(w, rows_check, heads=None):
