@@ -11,7 +11,11 @@ namespace abatt {
 struct Strides {
     int64_t sT, sH, sB;
     int H;
-    __host__ __device__ int64_t head_base(int64_t bh) const { return (bh / H) * sB + (bh % H) * sH; }
+    // bh = beta*H + h < 2^16 (B*H <= 65535 is a limit of the ABI): 32-bit division
+    __host__ __device__ int64_t head_base(int64_t bh) const {
+        const int b = (int)bh / H;
+        return b * sB + ((int)bh - b * H) * sH;
+    }
 };
 
 // ---- IBCS part 1: per-query-block k-means ---------------------------------
