@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="abatt", choices=["abatt", "reference"])
     ap.add_argument("--workload", default="wan14b-720p", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--sweep", action="store_true",
+                    help="the sweep workloads (H=24, N x budget x Bk): one JSON line per point, then a table")
+    ap.add_argument("--sweep-n", default=None, help="comma-separated subset of the sweep's N")
     ap.add_argument("--budget-bp", type=int, default=None, help="override (10000 = keep-all)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -80,6 +83,93 @@ def attention_traffic(rows: int):
     if not m or m.group(1) != hashlib.sha256(src).hexdigest()[:16]:
         return None
     return int(m.group(2)) * rows
+
+
+def run_sweep(args):
+    """Latency, tensor-pipe fraction and error of every sweep point (H=24,
+    d=128; N x budget x Bk) on one GPU.  The error is the relative L2 of O
+    against the same kernel in keep-all mode (budget 100 %: every block,
+    weight 1 -- dense attention, checked against the float64 oracle by the
+    GPU tests).  Inputs are drawn on the GPU (synth.generate_on_device)."""
+    import torch
+
+    from block_sparse_attention_20_b200 import abatt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pk, src = peaks()
+    peak = pk.get("bf16_tflops", FALLBACK_PEAK_TFLOPS)
+    Ns = synth.SWEEP_N if not args.sweep_n else tuple(int(x) for x in args.sweep_n.split(","))
+    reps = max(3, min(args.steps, 10))  # per sweep point
+    stream = torch.cuda.current_stream()
+    table = []
+    for N in Ns:
+        w0 = synth.sweep(N, 100, 16)
+        Q, K, V = synth.generate_on_device(w0, dev)
+        shape = w0.shape
+        for Bk in synth.SWEEP_BK:
+            O_ref = None
+            for bpct in sorted(synth.SWEEP_BUDGET, reverse=True):  # keep-all first: the reference
+                w = synth.sweep(N, bpct, Bk)
+                cfg = abatt.Config(kv_block=Bk, clusters=w.clusters, kmeans_iters=w.iters,
+                                   budget_bp=w.budget_bp, seed=w.seed)
+                rows, nK = w.rows, w.nK
+                p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
+                counts = torch.empty(rows, dtype=torch.int32, device=dev)
+                idx = torch.empty((rows, nK), dtype=torch.int32, device=dev)
+                logw = torch.empty((rows, nK), dtype=torch.float32, device=dev)
+                O = torch.empty_like(Q)
+                ws_sel = torch.empty(abatt.workspace_size(abatt.CALL_SELECT, shape, cfg), dtype=torch.uint8,
+                                     device=dev)
+                ws_small = torch.empty(256, dtype=torch.uint8, device=dev)
+                ws_att = torch.empty(abatt.workspace_size(abatt.CALL_ATTENTION, shape, cfg),
+                                     dtype=torch.uint8, device=dev)
+                ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+                for k in range(reps + 2):
+                    e = ev[k - 2] if k >= 2 else None
+                    if e: e[0].record(stream)
+                    abatt.select(Q, K, cfg, p=p, workspace=ws_sel, stream=stream)
+                    if e: e[1].record(stream)
+                    abatt.sample(p, shape, cfg, out=(counts, idx, logw), workspace=ws_small, stream=stream)
+                    if e: e[2].record(stream)
+                    abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws_att, stream=stream)
+                    if e: e[3].record(stream)
+                torch.cuda.synchronize()
+                status = abatt.read_status(ws_small) | abatt.read_status(ws_sel) | abatt.read_status(ws_att)
+                sel = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+                smp = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+                att = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
+                c = counts.cpu().numpy().astype(np.int64)
+                bpt = 128 // Bk
+                tiles = int(((c + bpt - 1) // bpt).sum())
+                exec_tf = tiles * 4.0 * 128 * 128 * w.d / (att * 1e-3) / 1e12
+                dense_flop = 4.0 * w.H * N * N * w.d
+                skip = 1.0 - float(np.minimum(c * Bk, N).sum()) / (w.H * w.nQ * N)
+                if O_ref is None:
+                    O_ref = O.float()
+                    err = 0.0
+                else:
+                    err = float((O.float() - O_ref).norm() / O_ref.norm())
+                rec = {"N": N, "kv_block": Bk, "budget_pct": bpct, "select_ms": sel, "sample_ms": smp,
+                       "attention_ms": att, "total_ms": sel + smp + att,
+                       "dense_equiv_tflops": dense_flop / ((sel + smp + att) * 1e-3) / 1e12,
+                       "executed_tflops_attention": exec_tf, "tensor_frac": exec_tf / peak,
+                       "realized_skip": skip, "rel_l2_vs_keep_all": err, "device_status": status}
+                print(json.dumps(rec), flush=True)
+                table.append(rec)
+                del p, counts, idx, logw, O, ws_sel, ws_att
+            del O_ref
+        del Q, K, V
+        torch.cuda.empty_cache()
+    print(f"\npeak {peak:.0f} TFLOP/s ({src} bf16 burst)")
+    print("| N | Bk | budget | select ms | sample ms | attention ms | total ms | dense-equiv TFLOP/s "
+          "| executed TFLOP/s | tensor frac | skip | rel L2 vs keep-all |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|---|")
+    for r in table:
+        print(f"| {r['N']} | {r['kv_block']} | {r['budget_pct']} % | {r['select_ms']:.2f} | {r['sample_ms']:.2f} "
+              f"| {r['attention_ms']:.2f} | {r['total_ms']:.2f} | {r['dense_equiv_tflops']:.0f} "
+              f"| {r['executed_tflops_attention']:.0f} | {r['tensor_frac']:.2f} | {r['realized_skip']:.3f} "
+              f"| {r['rel_l2_vs_keep_all']:.3f} |")
 
 
 def peaks():
@@ -241,6 +331,9 @@ def main():
         w = w.with_(budget_bp=args.budget_bp)
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
 
     import torch

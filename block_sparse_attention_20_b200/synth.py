@@ -154,6 +154,35 @@ def generate(w: Workload, heads=None):
     return tuple(x.view(1, nh, N, d) for x in out)
 
 
+def generate_on_device(w: Workload, device):
+    """The same prototype-Voronoi recipe as `generate`, drawn on the GPU with
+    torch's Philox generator (one stream per head, seeded from w.seed and the
+    head), for workloads too large to draw on the host in reasonable time.
+    Same distribution as `generate`, different numbers.  Returns [B, H, N, d]
+    bf16 device tensors."""
+    import torch
+
+    B, H, N, d, P = w.B, w.H, w.N, w.d, w.prototypes
+    coords = torch.from_numpy(token_coords(w.grid, N)).to(device=device, dtype=torch.float64)
+    out = [torch.empty((B * H, N, d), dtype=torch.bfloat16, device=device) for _ in range(3)]
+    for k in range(B * H):
+        g = torch.Generator(device=device)
+        g.manual_seed(int(w.seed) * 1000003 + k)
+        seeds = torch.rand((P, 3), generator=g, device=device, dtype=torch.float64)
+        proto = torch.randn((P, d), generator=g, device=device)
+        # nearest seed, ties to the smallest index (argmin returns the first)
+        near = torch.cdist(coords, seeds).argmin(dim=1)
+        pt = proto[near]
+        noise = float(w.noise)
+        q = pt + noise * torch.randn((N, d), generator=g, device=device)
+        kk = pt * (1.0 + 0.1 * torch.randn((N, d), generator=g, device=device))
+        kk += noise * torch.randn((N, d), generator=g, device=device)
+        v = torch.randn((N, d), generator=g, device=device)
+        for dst, src in zip(out, (q, kk, v)):
+            dst[k].copy_(src.to(torch.bfloat16))
+    return tuple(x.view(B, H, N, d) for x in out)
+
+
 def random_bf16(shape, seed: int, scale: float = 1.0):
     """Plain N(0, scale^2) bf16 tensor (for edge-case tests)."""
     import torch
