@@ -6,7 +6,8 @@
 // One CTA of 128 threads (4 warps) per query block.  The block's queries stay
 // in shared memory as bf16 (exact copies of the inputs).  Per round:
 //   - distances: ||c_j||^2 - 2 q.c_j, the dot products on the tensor cores
-//     (mma.sync m16n8k16, bf16 in, fp32 accumulate) with each fp32 centroid
+//     (mma.sync m16n8k16, bf16 in, fp32 accumulate; fragments by ldmatrix,
+//     the centroids' shared by a warp's two 16-row tiles) with each fp32 centroid
 //     split into a bf16 high part and a bf16 residual, so the products carry
 //     about 16 significant bits of the centroid; warp w takes rows
 //     32w..32w+31; the argmin (ties to the lower index) is reduced across the
@@ -51,6 +52,14 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void *row_
                  : "r"(smem_u32(row_addr)));
 }
 
+// four 8x8 b16 matrices as stored: lane l supplies the address of row l%8
+// of matrix l/8
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *row_addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(row_addr)));
+}
+
 // bf16 pair (lo, hi) of two 0/1 flags
 __device__ __forceinline__ uint32_t onehot_pair(bool lo, bool hi) {
     return (lo ? 0x3F80u : 0u) | (hi ? 0x3F800000u : 0u);
@@ -73,10 +82,6 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, cq = lane & 3;  // mma fragment coordinates
-    const uint32_t *qw = reinterpret_cast<const uint32_t *>(qs);
-    const uint32_t *hw = reinterpret_cast<const uint32_t *>(chi);
-    const uint32_t *lw = reinterpret_cast<const uint32_t *>(clo);
-    constexpr int LDW = LDQ / 2;  // row stride in 32-bit words
 
     for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
         const int i = (int)(row % a.nQ);
@@ -100,7 +105,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         __syncthreads();
         for (int e = tid; e < CP * D; e += kKmThreads) {
             const int j = e / D, x = e % D;
-            cent[e] = j < ce ? __bfloat162float(qs[(int)(((int64_t)j * n) / ce) * LDQ + x]) : 0.0f;
+            cent[e] = j < ce ? __bfloat162float(qs[(j * n) / ce * LDQ + x]) : 0.0f;
         }
         __syncthreads();
 
@@ -126,54 +131,69 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
             __syncthreads();
 
             // ---- assignment: q.c on tensor cores, argmin over centroids ----
+            // warp w: rows 32w..32w+31 as two 16-row MMA tiles; per 16-dim step one
+            // ldmatrix of each query tile and one of the centroids' hi and lo parts
+            // (shared by both tiles)
             const int nt = (ce + 7) >> 3;  // 8-wide centroid tiles
+            float bestd[2][2];
+            int besti[2][2];
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int r0 = warp * 32 + m * 16;
-                float bestd[2];
-                int besti[2];
+            for (int m = 0; m < 2; ++m)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) { bestd[h] = __int_as_float(0x7f800000); besti[h] = 0; }
-                for (int t = 0; t < nt; ++t) {
-                    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int h = 0; h < 2; ++h) { bestd[m][h] = __int_as_float(0x7f800000); besti[m][h] = 0; }
+            // lane roles in the x4 loads: query row (l % 16) at column half l / 16;
+            // centroid row (l % 8) of the hi (l < 16) or lo part at column half (l / 8) % 2
+            const __nv_bfloat16 *qa = qs + (warp * 32 + (lane & 15)) * LDQ + (lane >> 4) * 8;
+            for (int t = 0; t < nt; ++t) {
+                const __nv_bfloat16 *cb = (lane < 16 ? chi : clo) + (t * 8 + (lane & 7)) * LDQ + ((lane >> 3) & 1) * 8;
+                float acc[2][4];
 #pragma unroll
-                    for (int k0 = 0; k0 < D; k0 += 16) {
-                        const int kw = (k0 >> 1) + cq;  // word of column pair k0 + 2cq
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) acc[m][u] = 0.0f;
+#pragma unroll
+                for (int k0 = 0; k0 < D; k0 += 16) {
+                    uint32_t bf[4];  // hi (k0..7, k8..15), lo (k0..7, k8..15)
+                    ldsm_x4(bf, cb + k0);
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) {
                         uint32_t af[4];
-                        af[0] = qw[(r0 + g) * LDW + kw];
-                        af[1] = qw[(r0 + g + 8) * LDW + kw];
-                        af[2] = qw[(r0 + g) * LDW + kw + 4];
-                        af[3] = qw[(r0 + g + 8) * LDW + kw + 4];
-                        const int cj = t * 8 + g;
-                        mma_bf16_16816(acc, af, hw[cj * LDW + kw], hw[cj * LDW + kw + 4]);
-                        mma_bf16_16816(acc, af, lw[cj * LDW + kw], lw[cj * LDW + kw + 4]);
+                        ldsm_x4(af, qa + m * 16 * LDQ + k0);
+                        mma_bf16_16816(acc[m], af, bf[0], bf[1]);
+                        mma_bf16_16816(acc[m], af, bf[2], bf[3]);
                     }
-                    // acc[0..1]: row g, centroids t*8+2cq+{0,1}; acc[2..3]: row g+8
+                }
+                // acc[m][0..1]: row g, centroids t*8+2cq+{0,1}; acc[m][2..3]: row g+8
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int j = t * 8 + 2 * cq + u;
-                            const float dj = j < ce ? fmaf(-2.0f, acc[2 * h + u], cnorm[j])
+                            const float dj = j < ce ? fmaf(-2.0f, acc[m][2 * h + u], cnorm[j])
                                                     : __int_as_float(0x7f800000);
-                            if (dj < bestd[h]) { bestd[h] = dj; besti[h] = j; }
+                            if (dj < bestd[m][h]) { bestd[m][h] = dj; besti[m][h] = j; }
                         }
-                }
-                // combine the four lanes of each row (ties to the lower index)
+            }
+            // combine the four lanes of each row (ties to the lower index)
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int r0 = warp * 32 + m * 16;
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int o = 1; o < 4; o <<= 1) {
-                        const float od = __shfl_xor_sync(0xffffffffu, bestd[h], o);
-                        const int oi = __shfl_xor_sync(0xffffffffu, besti[h], o);
-                        if (od < bestd[h] || (od == bestd[h] && oi < besti[h])) {
-                            bestd[h] = od;
-                            besti[h] = oi;
+                        const float od = __shfl_xor_sync(0xffffffffu, bestd[m][h], o);
+                        const int oi = __shfl_xor_sync(0xffffffffu, besti[m][h], o);
+                        if (od < bestd[m][h] || (od == bestd[m][h] && oi < besti[m][h])) {
+                            bestd[m][h] = od;
+                            besti[m][h] = oi;
                         }
                     }
                 if (cq == 0) {
-                    assign_s[r0 + g] = (r0 + g) < n ? besti[0] : -1;
-                    assign_s[r0 + g + 8] = (r0 + g + 8) < n ? besti[1] : -1;
+                    assign_s[r0 + g] = (r0 + g) < n ? besti[m][0] : -1;
+                    assign_s[r0 + g + 8] = (r0 + g + 8) < n ? besti[m][1] : -1;
                 }
             }
             __syncthreads();
