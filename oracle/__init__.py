@@ -58,7 +58,7 @@ def _load():
         lib.orc_inclusion.argtypes = [P, i32, i64, P, P, P, P, P]
         lib.orc_topk.argtypes = [P, i64, i32, i32, i32, i32, P, P, P]
         lib.orc_sample.argtypes = [P, i32, i32, i32, i32, i32, P, i64, i32, u64, i32, i32,
-                                   P, P, P, P]
+                                   P, P, P, P, i32]
         lib.orc_ht_attention.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, i64,
                                          P, P, P, i32, i32, i32, P, P, P, P]
         lib.orc_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, i32, f64,
@@ -181,8 +181,12 @@ def inclusion(p_row, M):
     return P, sat.astype(bool), R.value, T.value, rounds.value
 
 
-def sample(p, shape, rows, budget_bp, seed, Bq=128, Bk=16, capacity=None, nthreads=None):
+def sample(p, shape, rows, budget_bp, seed, Bq=128, Bk=16, capacity=None, nthreads=None,
+           paired=False):
     """O4: SIP draw for the listed rows (p is fp32 [nrows, nK]).
+
+    paired=True: common random numbers -- query blocks 2j and 2j+1 of a head
+    draw with the same Philox counter (floor(i/2) in place of i).
 
     Returns counts [nrows], idx [nrows, cap], logw fp32 [nrows, cap],
     amb uint8 [nrows, cap] (1 where the fp32 rounding of -ln(pi) is too close
@@ -198,7 +202,8 @@ def sample(p, shape, rows, budget_bp, seed, Bq=128, Bk=16, capacity=None, nthrea
     amb = np.zeros((len(r), cap), dtype=np.uint8)
     rc = _check(_load().orc_sample(_ptr(p), B, H, N, Bq, Bk, _ptr(r), len(r), int(budget_bp),
                                    int(seed) & (2**64 - 1), cap, nthreads or default_threads(),
-                                   _ptr(counts), _ptr(idx), _ptr(logw), _ptr(amb)), "sample")
+                                   _ptr(counts), _ptr(idx), _ptr(logw), _ptr(amb), int(bool(paired))),
+                "sample")
     return counts, idx, logw, amb, bool(rc == 1)
 
 

@@ -525,6 +525,9 @@ int orc_block_probs(const uint16_t *Q, const uint16_t *K, int B, int H, int N, i
 /*     T = 0.  Outside S, pi_b = R*P_b / T exactly;                          */
 /*   - the draw for block b of row (beta,h,i) is word (b mod 4) of           */
 /*     Philox4x32-10 at counter (b/4, i, h, beta) and key (seed lo, seed hi);*/
+/*     with paired draws the counter is (b/4, floor(i/2), h, beta): query    */
+/*     blocks 2j and 2j+1 share every uniform (common random numbers; each   */
+/*     row keeps its own pi_b, so its marginal draws are unchanged);         */
 /*   - b is taken iff b is in S or U_b * T < R * P_b * 2^32 (exact integer  */
 /*     comparison, i.e. U_b / 2^32 < pi_b);                                  */
 /*   - log-weight: 0 on S, else fp32 round-to-nearest of -ln(x) with         */
@@ -603,7 +606,7 @@ static float neg_log_f32(double x, int *amb)
 }
 
 static int sample_row(const float *p, const geom_t *g, int beta, int h, int i,
-                      int budget_bp, uint64_t seed, int capacity,
+                      int budget_bp, uint64_t seed, int paired, int capacity,
                       int32_t *count, int32_t *idx, float *logw, uint8_t *amb,
                       int *overflow)
 {
@@ -620,7 +623,8 @@ static int sample_row(const float *p, const geom_t *g, int beta, int h, int i,
     *overflow = 0;
     for (int b = 0; b < nK; ++b) {
         if ((b & 3) == 0) {
-            const uint32_t ctr[4] = {(uint32_t)(b >> 2), (uint32_t)i, (uint32_t)h, (uint32_t)beta};
+            const uint32_t ctr[4] = {(uint32_t)(b >> 2), (uint32_t)(paired ? i >> 1 : i), (uint32_t)h,
+                                     (uint32_t)beta};
             orc_philox4x32_10(ctr, key, u4);
         }
         const uint32_t U = u4[b & 3];
@@ -654,7 +658,7 @@ typedef struct {
     const float *p;
     geom_t g;
     const int64_t *rows;
-    int budget_bp, capacity;
+    int budget_bp, capacity, paired;
     uint64_t seed;
     int32_t *counts, *idx;
     float *logw;
@@ -669,7 +673,7 @@ static void smp_row(void *vctx, int64_t k)
     if (decode_row(&c->g, c->rows[k], &beta, &h, &i)) { c->bad = 1; return; }
     size_t o = (size_t)k * c->capacity;
     if (sample_row(c->p + (size_t)k * c->g.nK, &c->g, beta, h, i, c->budget_bp, c->seed,
-                   c->capacity, c->counts + k, c->idx + o, c->logw + o,
+                   c->paired, c->capacity, c->counts + k, c->idx + o, c->logw + o,
                    c->amb ? c->amb + o : NULL, &of))
         c->bad = 1;
     if (of) __atomic_store_n(&c->overflow, 1, __ATOMIC_RELAXED);
@@ -680,7 +684,7 @@ static void smp_row(void *vctx, int64_t k)
 int orc_sample(const float *p, int B, int H, int N, int Bq, int Bk,
                const int64_t *rows, int64_t nrows, int budget_bp, uint64_t seed,
                int capacity, int nthreads,
-               int32_t *counts, int32_t *idx, float *logw, uint8_t *amb)
+               int32_t *counts, int32_t *idx, float *logw, uint8_t *amb, int paired)
 {
     smp_ctx c;
     memset(&c, 0, sizeof c);
@@ -688,7 +692,7 @@ int orc_sample(const float *p, int B, int H, int N, int Bq, int Bk,
     if (!p || !rows || !counts || !idx || !logw || capacity < 0 || budget_bp < 0) return -1;
     if (c.g.nK > 32767) return -1;
     c.p = p; c.rows = rows; c.budget_bp = budget_bp; c.capacity = capacity; c.seed = seed;
-    c.counts = counts; c.idx = idx; c.logw = logw; c.amb = amb;
+    c.counts = counts; c.idx = idx; c.logw = logw; c.amb = amb; c.paired = paired ? 1 : 0;
     parallel_for(nrows, nthreads, smp_row, &c);
     if (c.bad) return -2;
     return c.overflow ? 1 : 0;
@@ -923,7 +927,7 @@ static void fwd_row(void *vctx, int64_t k)
         c->bad = 1;
     } else {
         for (int b = 0; b < nK; ++b) p32[b] = (float)p[b];
-        if (sample_row(p32, g, beta, h, i, c->budget_bp, c->seed, nK, c->counts + k, idx,
+        if (sample_row(p32, g, beta, h, i, c->budget_bp, c->seed, 0, nK, c->counts + k, idx,
                        logw, NULL, &of))
             c->bad = 1;
         for (int s = 0; s < c->counts[k]; ++s) lwd[s] = (double)logw[s];

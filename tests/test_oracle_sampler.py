@@ -151,3 +151,67 @@ def test_capacity_truncates_and_flags():
     assert np.array_equal(cut[1][0], full[1][0, :L - 3])
     ok = oracle.sample(p, shape, [0], 5000, 1, capacity=L)
     assert not ok[4]
+
+
+# ---- paired draws (common random numbers across query blocks 2j, 2j+1) ----
+
+def test_paired_rows_with_equal_probabilities_draw_equal_lists():
+    # one uniform per (block, pair): equal p gives equal lists for the two rows
+    # of a pair, while independent draws give different ones
+    nK = 48
+    shape = (2, 3, nK * 16, 8)  # nQ = 6: pairs (0,1), (2,3), (4,5) per head
+    p = np.tile(synth.random_probs(1, nK, 21, 0.5), (36, 1))
+    rows = np.arange(36)
+    c, i, lw, _, _ = oracle.sample(p, shape, rows, 3000, 7, paired=True)
+    for r in range(0, 36, 2):
+        assert c[r] == c[r + 1] and np.array_equal(i[r, :c[r]], i[r + 1, :c[r]])
+        assert np.array_equal(lw[r, :c[r]], lw[r + 1, :c[r]])
+    ci, ii, _, _, _ = oracle.sample(p, shape, rows, 3000, 7)
+    assert sum(ci[r] != ci[r + 1] or not np.array_equal(ii[r, :ci[r]], ii[r + 1, :ci[r]])
+               for r in range(0, 36, 2)) >= 9
+    # different pairs still draw differently
+    assert len({tuple(i[r, :c[r]]) for r in range(0, 36, 2)}) > 12
+
+
+def test_paired_draw_of_a_row_is_the_independent_draw_at_half_its_index():
+    # under pairing, query blocks 2j and 2j+1 both draw with the counter that
+    # query block j has without it
+    nK = 40
+    shape = (1, 2, nK * 16, 8)  # nQ = 5 (the last pair has one row)
+    p = synth.random_probs(10, nK, 23, 0.3)
+    rows = np.arange(10)
+    cp, ip, lp, _, _ = oracle.sample(p, shape, rows, 2500, 11, paired=True)
+    for r in rows:
+        h, i = divmod(int(r), 5)
+        half = h * 5 + (i >> 1)
+        ce, ie, le, _, _ = oracle.sample(p[r:r + 1], shape, [half], 2500, 11)
+        assert cp[r] == ce[0] and np.array_equal(ip[r, :cp[r]], ie[0, :ce[0]])
+        assert np.array_equal(lp[r, :cp[r]], le[0, :ce[0]])
+
+
+def test_paired_draws_take_a_block_in_both_rows_with_the_smaller_probability():
+    # with one uniform U for both rows, block b is in both lists iff
+    # U < min(pi_0b, pi_1b): P(both) = min(pi_0b, pi_1b), against pi_0b*pi_1b
+    # for independent draws
+    nK, bp = 32, 2500  # M = 8
+    shape = (1, 1, nK * 16, 8)  # nQ = 2: one pair
+    p = synth.random_probs(2, nK, 29, 0.4)
+    M = oracle.budget_blocks(bp, nK)
+    pis = []
+    for r in range(2):
+        P, sat, R, T, _ = oracle.inclusion(p[r], M)
+        pis.append(np.array([float(x) for x in _oracle_pi([int(v) for v in P], sat, R, T)]))
+    nseed = 4000
+    both = np.zeros(nK)
+    for s in range(nseed):
+        c, i, _, _, _ = oracle.sample(p, shape, [0, 1], bp, s, paired=True)
+        both[np.intersect1d(i[0, :c[0]], i[1, :c[1]])] += 1
+    from scipy.stats import binom
+
+    want = np.minimum(pis[0], pis[1])
+    lo = binom.cdf(both, nseed, want)
+    hi = binom.sf(both - 1, nseed, want)
+    assert np.all(np.minimum(lo, hi) > 1e-7), (both, want * nseed)
+    # and not the independent rate where the two differ noticeably
+    gap = want - pis[0] * pis[1]
+    assert np.all(both[gap > 0.1] / nseed > (pis[0] * pis[1])[gap > 0.1] + 0.05)
