@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--e2e-heads", type=int, default=2, help="heads per chunk of the host pipeline")
     ap.add_argument("--selection", default="sip", choices=["sip", "topk"],
                     help="sip: the method's draw; topk: the truncating baseline")
+    ap.add_argument("--draws", default="independent", choices=["independent", "paired"],
+                    help="paired: query blocks 2j, 2j+1 share the sampler's uniforms")
     ap.add_argument("--scoring", default="keys", choices=["keys", "block-means"],
                     help="keys: every key scored (the method); block-means: the coarse baseline")
     return ap.parse_args()
@@ -359,7 +361,8 @@ def main():
                        batch_offset=plan["batch_offset"],
                        selection=abatt.SELECT_TOPK if args.selection == "topk" else abatt.SELECT_SIP,
                        scoring=(abatt.SCORE_BLOCK_MEANS if args.scoring == "block-means"
-                                else abatt.SCORE_KEYS))
+                                else abatt.SCORE_KEYS),
+                       draws=abatt.DRAWS_PAIRED if args.draws == "paired" else abatt.DRAWS_INDEPENDENT)
     rows, nK = w.rows, w.nK
     p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
     counts = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -432,6 +435,16 @@ def main():
     pk, src = peaks()
     peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
     achieved = alg_flop / (att_mean * 1e-3) / 1e12
+    # blocks the two rows of a pair both drew (gathered once for both), over
+    # the blocks either drew
+    both = either = 0
+    for r in range(0, rows - 1, 2):
+        if (r % w.nQ) % 2 or r // w.nQ != (r + 1) // w.nQ:
+            continue
+        a0, a1 = idx_h[r, :c[r]], idx_h[r + 1, :c[r + 1]]
+        k = np.intersect1d(a0, a1, assume_unique=True).size
+        both += k
+        either += a0.size + a1.size - k
 
     line = {
         "metric": METRIC,
@@ -443,13 +456,14 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters,
                    "kmeans_iters": w.iters, "selection": args.selection,
-                   "scoring": args.scoring,
+                   "scoring": args.scoring, "draws": args.draws,
                    "per_rank": "one batch element per GPU",
                    "l2": "inputs (Q,K,V 2.3 GB) exceed the 126 MB L2; no flush"},
         "stages_ms": {"select": sel_ms, "sample": smp_ms, "attention": att_ms},
         "attention_ms": att_ms,
         "selector_sampler_share": (sel_ms + smp_ms) / (sel_ms + smp_ms + att_ms),
         "realized_skip": skip,
+        "pair_shared_fraction": both / max(either, 1),
         "executed_tflops_attention": exec_flop / (att_mean * 1e-3) / 1e12,
         "algorithmic_tflops_attention": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

@@ -23,6 +23,7 @@ CALL_SELECT, CALL_SAMPLE, CALL_ATTENTION, CALL_FORWARD = 0, 1, 2, 3
 SELECT_SIP, SELECT_TOPK = 0, 1
 SCORE_KEYS, SCORE_BLOCK_MEANS = 0, 1
 LAYOUT_BHND, LAYOUT_BNHD = 0, 1
+DRAWS_INDEPENDENT, DRAWS_PAIRED = 0, 1
 DEVFLAG_CAPACITY, DEVFLAG_TIMEOUT, DEVFLAG_BADLIST = 0x1, 0x2, 0x4
 
 # Every symbol declared in include/abatt.h.
@@ -49,7 +50,7 @@ class _Config(ctypes.Structure):
                 ("scale", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("batch_offset", ctypes.c_int), ("head_offset", ctypes.c_int),
                 ("selection", ctypes.c_int), ("scoring", ctypes.c_int),
-                ("layout", ctypes.c_int), ("reserved", ctypes.c_int)]
+                ("layout", ctypes.c_int), ("draws", ctypes.c_int)]
 
 
 @dataclass(frozen=True)
@@ -68,12 +69,13 @@ class Config:
     selection: int = 0     # SELECT_SIP (the method) or SELECT_TOPK (truncating baseline)
     scoring: int = 0       # SCORE_KEYS (the method as read) or SCORE_BLOCK_MEANS (coarse baseline)
     layout: int = 0        # LAYOUT_BHND ([B,H,N,d]) or LAYOUT_BNHD ([B,N,H,d])
+    draws: int = 0         # DRAWS_INDEPENDENT or DRAWS_PAIRED (query blocks 2j, 2j+1 share uniforms)
 
     def _c(self, d: int) -> _Config:
         s = self.scale if self.scale is not None else 1.0 / math.sqrt(d)
         return _Config(self.q_block, self.kv_block, self.clusters, self.kmeans_iters,
                        self.budget_bp, s, self.seed & (2**64 - 1), self.batch_offset, self.head_offset,
-                       self.selection, self.scoring, self.layout, 0)
+                       self.selection, self.scoring, self.layout, self.draws)
 
 
 _lock = threading.Lock()

@@ -70,6 +70,7 @@ abatt_status validate(const abatt_shape *s, const abatt_config *c, Geom *g) {
     if (c->selection != ABATT_SELECT_SIP && c->selection != ABATT_SELECT_TOPK) return ABATT_ERR_INVALID_ARG;
     if (c->scoring != ABATT_SCORE_KEYS && c->scoring != ABATT_SCORE_BLOCK_MEANS) return ABATT_ERR_INVALID_ARG;
     if (c->layout != ABATT_LAYOUT_BHND && c->layout != ABATT_LAYOUT_BNHD) return ABATT_ERR_INVALID_ARG;
+    if (c->draws != ABATT_DRAWS_INDEPENDENT && c->draws != ABATT_DRAWS_PAIRED) return ABATT_ERR_INVALID_ARG;
     if (s->d != 64 && s->d != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->q_block != 128) return ABATT_ERR_UNSUPPORTED;
     if (c->kv_block != 16 && c->kv_block != 32 && c->kv_block != 64 && c->kv_block != 128)
@@ -291,6 +292,7 @@ abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, 
     a.p = p; a.rows = g.rows; a.nK = g.nK; a.nK_pad = (g.nK + 3) & ~3; a.nQ = g.nQ; a.H = g.H;
     a.M = g.M;
     a.topk = cfg->selection == ABATT_SELECT_TOPK ? 1 : 0;
+    a.paired = cfg->draws == ABATT_DRAWS_PAIRED ? 1 : 0;
     a.b_off = (uint32_t)cfg->batch_offset;
     a.h_off = (uint32_t)cfg->head_offset;
     a.key0 = (uint32_t)(cfg->seed & 0xffffffffu);

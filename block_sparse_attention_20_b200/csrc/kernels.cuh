@@ -103,6 +103,7 @@ struct SampleArgs {
     int64_t M;
     uint32_t b_off, h_off;  // global index of the first batch element / head (Philox counter)
     int topk;               // 1: keep the M largest estimates (weight 1) instead of drawing
+    int paired;             // 1: Philox counter word 1 is i/2 (query blocks 2j, 2j+1 share draws)
     uint32_t key0, key1;
     int capacity;
     int32_t *counts, *idx;

@@ -168,8 +168,9 @@ __global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleAr
             uint64_t rp[4] = {0, 0, 0, 0};
             int cnt = 0;
             if (b0 < nK) {
-                const uint4 u = philox4x32_10(
-                    make_uint4((uint32_t)g, (uint32_t)i, (uint32_t)h + a.h_off, (uint32_t)beta + a.b_off), a.key0, a.key1);
+                const uint4 u = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(a.paired ? i >> 1 : i),
+                                                         (uint32_t)h + a.h_off, (uint32_t)beta + a.b_off),
+                                              a.key0, a.key1);
                 const uint32_t U[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -428,7 +429,9 @@ __global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
             const int g = tid * G + u;
             if (4 * g >= nK) break;
             const uint4 r4 =
-                philox4x32_10(make_uint4((uint32_t)g, (uint32_t)i, (uint32_t)h + a.h_off, (uint32_t)beta + a.b_off), a.key0, a.key1);
+                philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(a.paired ? i >> 1 : i), (uint32_t)h + a.h_off,
+                                         (uint32_t)beta + a.b_off),
+                              a.key0, a.key1);
             const uint32_t U[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

@@ -78,6 +78,17 @@ typedef struct abatt_shape {
         (ABATT_ERR_UNSUPPORTED otherwise). */
 enum { ABATT_SELECT_SIP = 0, ABATT_SELECT_TOPK = 1 };
 
+/* Where the sampler's uniforms come from.
+   INDEPENDENT: Philox counter (b/4, i, h, beta) -- every query block draws on
+        its own (the method as read).
+   PAIRED: counter (b/4, floor(i/2), h, beta) -- query blocks 2j and 2j+1 of a
+        head share every uniform (common random numbers).  Each row keeps its
+        own inclusion probabilities, so its draw is marginally the same Poisson
+        sample and its estimate stays unbiased; a block lands in both lists with
+        probability min(pi_0, pi_1) instead of pi_0*pi_1, so the two rows, which
+        abatt_attention processes together, gather more blocks once for both. */
+enum { ABATT_DRAWS_INDEPENDENT = 0, ABATT_DRAWS_PAIRED = 1 };
+
 /* Memory layout of Q, K, V and O.
    BHND: [B][H][N][d] -- each head's tokens contiguous.
    BNHD: [B][N][H][d] -- token-major with the heads interleaved, as the
@@ -109,7 +120,7 @@ typedef struct abatt_config {
     int selection;      /* ABATT_SELECT_SIP (0, the method) or ABATT_SELECT_TOPK (1) */
     int scoring;        /* ABATT_SCORE_KEYS (0, the method as read) or ABATT_SCORE_BLOCK_MEANS (1) */
     int layout;         /* ABATT_LAYOUT_BHND (0) or ABATT_LAYOUT_BNHD (1) */
-    int reserved;       /* set to 0 */
+    int draws;          /* ABATT_DRAWS_INDEPENDENT (0) or ABATT_DRAWS_PAIRED (1) */
     /* The sampler's Philox counter uses the global indices (beta + batch_offset,
        h + head_offset), so a call over a slice of the batches or heads of a
        larger problem draws exactly the blocks that one call over the whole
@@ -148,7 +159,8 @@ abatt_status abatt_select(const void *Q, const void *K, const abatt_shape *shape
  * inclusion probabilities pi_b = min(1, c p_b), sum_b pi_b = M, solved
  * exactly in 48-bit fixed point (P_b = round-half-even(p_b 2^48), p clamped
  * to [0,1], NaN read as 0; water-filling of the saturated set).  Draw U_b is
- * word (b mod 4) of Philox4x32-10 at counter (b/4, i, h, beta), key
+ * word (b mod 4) of Philox4x32-10 at counter (b/4, i, h, beta) (i/2 in
+ * place of i with ABATT_DRAWS_PAIRED), key
  * (seed lo, seed hi); block b is taken iff saturated or U_b/2^32 < pi_b
  * (exact integer test).
  * Outputs: counts int32 [rows]; idx int32 [rows][capacity] in ascending

@@ -76,6 +76,7 @@ def test_workspace_sizes():
     ((1, 1, 100, 64), {"selection": 2}, 1),
     ((1, 1, 100, 64), {"scoring": 3}, 1),
     ((1, 1, 100, 64), {"layout": 2}, 1),
+    ((1, 1, 100, 64), {"draws": 2}, 1),
     ((1, 1, 16 * 10241, 64), {"selection": 1}, 2),   # top-M needs nK <= 10240
 ])
 def test_validation(shape, kw, code):
@@ -130,5 +131,5 @@ def test_config_struct_carries_the_slice_offsets():
     assert ctypes.sizeof(c) == 56
     assert (c.seed, c.batch_offset, c.head_offset) == (5, 2, 7)
     assert abatt._Config.selection.offset == 40 and abatt._Config.scoring.offset == 44
-    assert abatt._Config.layout.offset == 48 and abatt._Config.reserved.offset == 52
+    assert abatt._Config.layout.offset == 48 and abatt._Config.draws.offset == 52
     assert abatt._Config.head_offset.offset == 36 and abatt._Config.batch_offset.offset == 32

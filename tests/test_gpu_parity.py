@@ -120,6 +120,21 @@ def test_sample_topk_bit_exact(nK, bp, coarse):
         assert np.all(lw[r, :c[r]] == 0)
 
 
+@pytest.mark.parametrize("nK,Bk,bp", [(256, 16, 1000), (4725, 16, 800), (7425, 16, 1100), (10300, 16, 700),
+                                      (63, 16, 2500)])
+def test_sample_paired_bit_exact(nK, Bk, bp):
+    # common random numbers: the counter's query-block word is i/2
+    N = nK * Bk - Bk // 2
+    shape = (1, 2, N, 64)
+    rows = _rows_of(shape)
+    p = synth.random_probs(len(rows), nK, 3000 + nK, 0.2)
+    cfg = abatt.Config(kv_block=Bk, budget_bp=bp, seed=0x1234ABCD5678EF90, draws=abatt.DRAWS_PAIRED)
+    c, i, lw, ws = abatt.sample(torch.from_numpy(p).cuda(), shape, cfg)
+    assert abatt.read_status(ws) == 0
+    oc, oi, ol, oamb, _ = oracle.sample(p, shape, rows, bp, cfg.seed, Bk=Bk, paired=True)
+    _check_lists_exact(c.cpu().numpy(), i.cpu().numpy(), lw.cpu().numpy(), oc, oi, ol, oamb)
+
+
 def test_sample_capacity_overflow_flags_and_truncates():
     nK, Bk = 512, 16
     shape = (1, 1, nK * Bk, 64)
@@ -400,6 +415,50 @@ def test_forward_block_means_tiny():
         got[r] = Oc[0, h, q * 128:(q + 1) * 128]
     assert _rel_l2(got, o5) <= REL_L2
     assert np.max(np.abs(got - o5)) <= MAX_ABS
+
+
+def _pair_overlap(counts, idx, nQ):
+    # mean |S_2j & S_2j+1| / |S_2j | S_2j+1| over the pairs of every head
+    fr = []
+    for r in range(0, len(counts) - 1, 2):
+        if r // nQ != (r + 1) // nQ or (r % nQ) % 2:
+            continue
+        a_, b_ = set(idx[r, :counts[r]].tolist()), set(idx[r + 1, :counts[r + 1]].tolist())
+        if a_ | b_:
+            fr.append(len(a_ & b_) / len(a_ | b_))
+    return float(np.mean(fr))
+
+
+def test_forward_paired_draws():
+    # paired draws end to end: lists bit-exact against the oracle's paired
+    # sampler on the kernel's own p, attention on them, and a pair's two lists
+    # overlap more than with independent draws
+    w = synth.WAN_1_3B.with_(H=2)
+    Q, K, V = synth.generate(w)
+    shape = w.shape
+    res = {}
+    for mode in (abatt.DRAWS_INDEPENDENT, abatt.DRAWS_PAIRED):
+        cfg = cfg_of(w, draws=mode)
+        ws = torch.empty(abatt.workspace_size(abatt.CALL_FORWARD, shape, cfg), dtype=torch.uint8,
+                         device="cuda")
+        O = abatt.forward(Q.cuda(), K.cuda(), V.cuda(), cfg, workspace=ws)
+        torch.cuda.synchronize()
+        assert abatt.read_status(ws) == 0
+        res[mode] = (O.float().cpu().numpy(), *(t.cpu().numpy() for t in abatt.intermediates(ws, shape, cfg)))
+    O, p, counts, idx, logw = res[abatt.DRAWS_PAIRED]
+    rows = _rows_of(shape)
+    oc, oi, ol, oamb, _ = oracle.sample(p, shape, rows, w.budget_bp, w.seed, Bk=w.Bk, paired=True)
+    _check_lists_exact(counts, idx, logw, oc, oi, ol, oamb)
+    sub = rows[::16]
+    o5, _ = oracle.ht_attention(Q, K, V, shape, sub, counts[sub], idx[sub], logw[sub], Bk=w.Bk)
+    got = np.zeros_like(o5)
+    for k, r in enumerate(sub):
+        h, q = divmod(int(r), w.nQ)
+        n = min(128, w.N - q * 128)
+        got[k, :n] = O[0, h, q * 128:q * 128 + n]
+    assert _rel_l2(got, o5) <= REL_L2
+    ind = res[abatt.DRAWS_INDEPENDENT]
+    assert _pair_overlap(counts, idx, w.nQ) > _pair_overlap(ind[2], ind[3], w.nQ) + 0.05
 
 
 # ------------------------------------------------------------------- [B, N, H, d] layout
