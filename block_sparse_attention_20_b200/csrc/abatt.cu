@@ -124,7 +124,7 @@ Layout layout(abatt_call call, const Geom &g) {
         const size_t pairs = (size_t)pairs_of(g);
         L.useg = off; off = align256(off + pairs * 16);
         L.ublk = off; off = align256(off + pairs * g.nK * 4);
-        L.ulw = off;  off = align256(off + pairs * 2 * g.nK * 4);
+        L.ulw = off;  off = align256(off + pairs * 2 * (size_t)((g.nK + 7) & ~7) * 4);
     }
     if (call == ABATT_CALL_FORWARD) {
         L.p = off;      off = align256(off + (size_t)g.rows * g.nK * 4);
@@ -310,6 +310,9 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     PairArgs pa;
     pa.rows = g.rows; pa.pairs = pairs_of(g); pa.nQ = g.nQ; pa.nK = g.nK; pa.capacity = capacity; pa.cap_u = g.nK;
     pa.counts = counts; pa.idx = idx; pa.logw = logw;
+    pa.ragged = (g.N % g.Bk) != 0 ? 1 : 0;
+    pa.bpt = 128 / g.Bk;
+    pa.cap_w = (g.nK + 7) & ~7;
     pa.useg = at<int32_t>(ws, L.useg);
     pa.ublk = at<int32_t>(ws, L.ublk);
     pa.ulw = at<float>(ws, L.ulw);
@@ -351,7 +354,7 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     }
     AttnArgs a;
     a.rows = g.rows; a.pairs = pairs_of(g); a.nQ = g.nQ; a.N = g.N; a.D = g.d; a.Bk = g.Bk;
-    a.nK = g.nK; a.cap_u = g.nK; a.k_fold = fold ? 1 : 0;
+    a.nK = g.nK; a.cap_u = g.nK; a.cap_w = pa.cap_w; a.k_fold = fold ? 1 : 0;
     a.kf_gb = bnhd ? g.N / 8 : 0;
     a.kf_zb = bnhd ? 0 : g.H;
     a.st = sd;

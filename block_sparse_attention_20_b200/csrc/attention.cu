@@ -78,6 +78,8 @@ __global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArg
     // the three segment counts (both rows, row 0 only, row 1 only)
     extern __shared__ uint32_t sm_union[];
     __shared__ uint64_t wsum[kUnionThreads / 32];
+    __shared__ int tail_pos_s;  // position of the partial last key block in the pair's array
+    const bool ragged = a.ragged != 0;
     const int W = (a.nK + 31) >> 5;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t *bA = sm_union, *bB = sm_union + W;
@@ -85,6 +87,7 @@ __global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArg
     for (int64_t pr = blockIdx.x; pr < a.pairs; pr += gridDim.x) {
         __syncthreads();
         for (int w = tid; w < 2 * W; w += kUnionThreads) sm_union[w] = 0;
+        if (tid == 0) tail_pos_s = -1;
         __syncthreads();
         int64_t rr[2];
         pair_rows(pr, a.nQ, &rr[0], &rr[1]);
@@ -144,13 +147,17 @@ __global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArg
             for (int q = 0; q < 3; ++q) {
                 int pos = base[q];
                 for (uint32_t mu = seg[q]; mu; mu &= mu - 1) {
-                    if (pos < a.cap_u) ub[pos] = w * 32 + __ffs(mu) - 1;
+                    const int k = w * 32 + __ffs(mu) - 1;
+                    if (pos < a.cap_u) ub[pos] = k;
+                    if (ragged && k == a.nK - 1) tail_pos_s = pos;
                     ++pos;
                 }
             }
         }
-        // each valid drawn entry writes its row's log-weight at its position
-        float *uw = a.ulw + pr * 2 * (int64_t)a.cap_u;
+        // each valid drawn entry writes its row's base-2 log-weight at its index
+        // in the row's sequence (row 0: [both | row 0 only] = positions 0..;
+        // row 1: [both | row 1 only], its own segment na positions earlier)
+        float *uw = a.ulw + pr * 2 * (int64_t)a.cap_w;
         for (int s = 0; s < 2; ++s) {
             const int32_t *idx = a.idx + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
             const float *lw = a.logw + (rr[s] >= 0 ? rr[s] : 0) * (int64_t)a.capacity;
@@ -163,14 +170,21 @@ __global__ void __launch_bounds__(kUnionThreads) pair_union_kernel(const PairArg
                 int pos;
                 if ((xa & xb) >> (k & 31) & 1u) pos = (int)preB[w] + __popc(xa & xb & below);
                 else if (s == 0) pos = nb + (int)preA[w] + __popc(xa & ~xb & below);
-                else pos = nb + na + (int)preC[w] + __popc(xb & ~xa & below);
-                if (pos < a.cap_u) uw[s * a.cap_u + pos] = lw[j];
+                else pos = nb + (int)preC[w] + __popc(xb & ~xa & below);
+                if (pos < a.cap_u) uw[s * a.cap_w + pos] = lw[j] * kLog2e;
             }
+            // -inf after the sequence up to the end of its last tile: the
+            // attention kernel reads whole tiles of weights
+            const int U = rr[s] >= 0 ? (s == 0 ? nb + na : nb + nc) : 0;
+            const int Upad = (U + a.bpt - 1) / a.bpt * a.bpt;
+            if (tid < Upad - U && U + tid < a.cap_w) uw[s * a.cap_w + U + tid] = kNegInf;
         }
+        __syncthreads();  // tail_pos_s is written
         if (tid == 0) {
             a.useg[pr * 4 + 0] = nb;
             a.useg[pr * 4 + 1] = na;
             a.useg[pr * 4 + 2] = nc;
+            a.useg[pr * 4 + 3] = tail_pos_s;
         }
     }
 }
@@ -488,42 +502,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int i = (int)(row % a.nQ), hd = (int)(row / a.nQ);
             const int nrows = min(128, a.N - i * 128);
             const int64_t tok = (int64_t)hd * a.N + (int64_t)i * 128 + r;
-            const int32_t *ub = a.ublk + pr * (int64_t)a.cap_u;
-            const float *lw = a.ulw + (pr * 2 + s) * (int64_t)a.cap_u;
+            const float *lw = a.ulw + (pr * 2 + s) * (int64_t)a.cap_w;
             float m_run = kNegInf, l = 0.0f;
-            // raw log-weights and block ids of this half's blocks for the next
-            // tile, loaded one tile ahead and first read at that tile (their
-            // latency hides behind the current tile)
+            // entry of this row's sequence that holds the partial last key
+            // block (-1: none): its keys past N are masked
+            const int tp = a.useg[pr * 4 + 3];
+            const int etail = tp < 0 ? -1
+                              : s == 0 ? (tp < P.nb + P.na ? tp : -1)
+                                       : (tp < P.nb ? tp : (tp >= P.nb + P.na ? tp - P.na : -1));
+            const int tail_keep = a.N - (a.nK - 1) * BK;
+            // base-2 log-weights of this half's blocks for the next tile (the
+            // row's sequence, -inf past its end), one vector load one tile ahead,
+            // first read at that tile (its latency hides behind the current tile)
             float nw[HB];
-            int nbk[HB];
             auto load_meta = [&](int t) {
-#pragma unroll
-                for (int k = 0; k < HB; ++k) {
-                    const int e = t * BPT + (BPT >= 2 ? hh * HB + k : 0);
-                    nw[k] = -1.0f;  // empty slot: not drawn
-                    nbk[k] = 0;
-                    if (e < U) {
-                        const int j = P.pos(s, e);
-                        nw[k] = __ldg(lw + j);
-                        nbk[k] = __ldg(ub + j);
-                    }
+                const float *src = lw + t * BPT + (BPT >= 2 ? hh * HB : 0);
+                if constexpr (HB == 4) {
+                    const float4 q = __ldg(reinterpret_cast<const float4 *>(src));
+                    nw[0] = q.x; nw[1] = q.y; nw[2] = q.z; nw[3] = q.w;
+                } else if constexpr (HB == 2) {
+                    const float2 q = __ldg(reinterpret_cast<const float2 *>(src));
+                    nw[0] = q.x; nw[1] = q.y;
+                } else {
+                    nw[0] = __ldg(src);
                 }
             };
             if (n > 0) load_meta(0);
             for (int t = 0; t < n; ++t) {
-                // this half's blocks: base-2 log-weight (-inf where this row did
-                // not draw the block or the slot is empty); the block that can
-                // be cut by N is the last block of the sequence
                 float bias[HB];
-                int tail_k = -1, tail_keep = BK;
 #pragma unroll
-                for (int k = 0; k < HB; ++k) {
-                    const float w = nw[k];
-                    const int b = nbk[k];
-                    bias[k] = w >= 0.0f ? w * kLog2e : kNegInf;
-                    if (w >= 0.0f && b == a.nK - 1 && a.N - b * BK < BK) {
-                        tail_k = k;
-                        tail_keep = a.N - b * BK;
+                for (int k = 0; k < HB; ++k) bias[k] = nw[k];
+                int tail_k = -1;
+                {
+                    const int et = etail - t * BPT;  // the tail block's slot in this tile
+                    if (et >= 0 && et < BPT) {
+                        const int k = BPT >= 2 ? et - hh * HB : 0;
+                        if (k >= 0 && k < HB) tail_k = k;
                     }
                 }
                 if (t + 1 < n) load_meta(t + 1);

@@ -135,11 +135,15 @@ __host__ __device__ __forceinline__ void pair_rows(int64_t pr, int nQ, int64_t *
 struct PairArgs {
     int64_t rows, pairs;
     int nQ, nK, capacity, cap_u;
+    int ragged;     // N % Bk != 0: the last key block is partial
+    int bpt;        // key blocks per 128-key tile
+    int cap_w;      // row stride of ulw (nK rounded up to 8)
     const int32_t *counts, *idx;
     const float *logw;
-    int32_t *useg;  // [pairs][4]       nb, na, nc (segment lengths), unused
+    int32_t *useg;  // [pairs][4]       nb, na, nc (segment lengths), position of a partial last block (-1: none)
     int32_t *ublk;  // [pairs][cap_u]   [both | row 0 only | row 1 only], ascending within each
-    float *ulw;     // [pairs][2][cap_u] row s's log-weight at the positions of its blocks
+    float *ulw;     // [pairs][2][cap_w] row s's log-weights in base 2 (log2(e) * -ln pi) in the order of its
+                    // sequence ([both | own]), -inf up to its last tile's end
     uint32_t *status;
 };
 cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t stream);
@@ -147,7 +151,7 @@ cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t strea
 struct AttnArgs {
     int64_t rows, pairs;  // query blocks, row pairs
     int nQ, N, D, Bk, nK;
-    int cap_u;
+    int cap_u, cap_w;
     int k_fold;        // K tiles as boxes of 8-row groups (needs N % 8 == 0)
     int kf_gb, kf_zb;  // k_fold: group coordinate b*kf_gb + blk*Bk/8, outer coordinate b*kf_zb + h
     Strides st;        // of O (and of Q, K, V in the maps)
