@@ -133,3 +133,21 @@ def test_config_struct_carries_the_slice_offsets():
     assert abatt._Config.selection.offset == 40 and abatt._Config.scoring.offset == 44
     assert abatt._Config.layout.offset == 48 and abatt._Config.draws.offset == 52
     assert abatt._Config.head_offset.offset == 36 and abatt._Config.batch_offset.offset == 32
+
+
+def test_host_pipeline_streams_head_chunks_of_bhnd_only():
+    # head chunks of a [B, N, H, d] tensor are not contiguous: refused before
+    # any device allocation
+    cfg = abatt.Config(layout=abatt.LAYOUT_BNHD)
+    with pytest.raises(ValueError):
+        abatt.HostPipeline((1, 4, 1024, 64), cfg)
+
+
+def test_shape_of_follows_the_layout():
+    import torch
+
+    q = torch.empty((2, 300, 5, 64))
+    sh = abatt._shape_of(q, abatt.Config(layout=abatt.LAYOUT_BNHD))
+    assert (sh.B, sh.H, sh.N, sh.d) == (2, 5, 300, 64)
+    sh = abatt._shape_of(q, abatt.Config())
+    assert (sh.B, sh.H, sh.N, sh.d) == (2, 300, 5, 64)
