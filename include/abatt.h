@@ -124,7 +124,9 @@ typedef struct abatt_config {
     /* The sampler's Philox counter uses the global indices (beta + batch_offset,
        h + head_offset), so a call over a slice of the batches or heads of a
        larger problem draws exactly the blocks that one call over the whole
-       problem draws for that slice.  Both must be >= 0 (ABATT_ERR_INVALID_ARG). */
+       problem draws for that slice.  Both must be >= 0 (ABATT_ERR_INVALID_ARG).
+       selection, scoring, layout and draws outside their listed values also
+       return ABATT_ERR_INVALID_ARG, before any launch. */
 } abatt_config;
 
 /* Which call a workspace is for. */
