@@ -367,9 +367,8 @@ def test_select_block_means_tiny():
                                     (20000, 64, 16), (3000, 32, 1), (3000, 16, 2), (20000, 16, 4)])
 def test_select_block_means_ragged(N, Bk, C):
     # partial last blocks (the n_b weight), several 128-block column tiles with a
-    # ragged last one, and (at 20000 keys) key ranges split over chunks; C that
-    # divides 32 takes the two-pass path that sums centroid lanes, C = 3 and 5
-    # the path through the block-value matrix
+    # ragged last one; C that divides 32 takes the two-pass path that sums
+    # centroid lanes, C = 3 and 5 the path through the block-value matrix
     w = synth.WAN_1_3B.with_(H=2, N=N, grid=(1, 20, N // 20))
     Q, K, V = synth.generate(w)
     _select_check(Q, K, w.shape, C, 5, Bk, coarse=True)
