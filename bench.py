@@ -293,10 +293,18 @@ def cpu_baseline(w, Q, K, V, budget_s=15.0):
     dt = time.perf_counter() - t0
     full = dt * w.rows / len(rows)
     dense = 4.0 * w.B * w.H * w.N * w.N * w.d
+    # and the whole tiny workload (every query block) on one thread
+    tw = synth.TINY
+    Qt, Kt, Vt = synth.generate(tw)
+    t0 = time.perf_counter()
+    oracle.forward(Qt, Kt, Vt, tw.shape, np.arange(tw.rows), tw.clusters, tw.iters, tw.budget_bp, tw.seed,
+                   Bk=tw.Bk, nthreads=1)
+    dt1 = time.perf_counter() - t0
     return {"value": dense / full / 1e12, "unit": "TFLOPS (dense-equivalent)", "cores": cores,
             "kind": "oracle",
             "sample": f"{len(rows)} of {w.rows} query blocks (every {stride}th), {dt:.1f} s, "
-                      f"extrapolated x{w.rows / len(rows):.1f}"}
+                      f"extrapolated x{w.rows / len(rows):.1f}",
+            "tiny_one_thread_s": dt1}
 
 
 def rank_plan(w, rank: int, world: int) -> dict:
