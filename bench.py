@@ -487,7 +487,7 @@ def main():
         line["keep_all"] = keep_all(abatt, cfg, Q, K, V, w, O, ws_att, stream)
     if not args.no_e2e:
         line["e2e"] = e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world)
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the host baseline: one process alone
         line["cpu_baseline"] = cpu_baseline(w, Qc, Kc, Vc)
     if rank == 0:
         print(json.dumps(line), flush=True)
