@@ -10,7 +10,9 @@ Prints one JSON line (rank 0).  `value` is dense-equivalent TFLOPS
 (4 B H N^2 d per step / step time) summed over ranks; the roofline object
 covers the gather-attention kernel (executed 128x128 tiles, tensor bound).
 With N > 1 GPUs (torchrun), every rank runs its own batch element (heads are
-independent; no collective on the data path): weak scaling.
+independent; no collective on the data path): weak scaling; with
+`--split heads` the ranks share out the heads of the one problem instead
+(strong scaling).
 """
 from __future__ import annotations
 
@@ -34,7 +36,7 @@ METRIC = "attention ms & dense-equiv TFLOPS at 90% skip; % bf16 tensor peak (1 B
 FALLBACK_PEAK_TFLOPS = 1590.0
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
@@ -55,7 +57,10 @@ def parse():
                     help="paired: query blocks 2j, 2j+1 share the sampler's uniforms")
     ap.add_argument("--scoring", default="keys", choices=["keys", "block-means"],
                     help="keys: every key scored (the method); block-means: the coarse baseline")
-    return ap.parse_args()
+    ap.add_argument("--split", default="batch", choices=["batch", "heads"],
+                    help="N > 1: batch -- one batch element per GPU (weak scaling); heads -- the "
+                         "heads of one problem shared out over the GPUs (strong scaling)")
+    return ap.parse_args(argv)
 
 
 def attention_source(csrc: str) -> bytes:
@@ -66,25 +71,28 @@ def attention_source(csrc: str) -> bytes:
         (head[cut:] if cut >= 0 else head)
 
 
-def attention_traffic(rows: int):
-    """DRAM bytes of one gather_attn_kernel launch, from the committed ncu
-    summary (bytes per query block, scaled by the launch's query blocks; DRAM
-    traffic of the kernel is its compulsory Q/K/V/O bytes, which grow with the
-    query blocks).  None when the kernel source differs from the one the
-    counters were taken on: attention.cu, common.cuh and the gather-attention
-    part of kernels.cuh (from its "---- gather attention" heading on)."""
+TRAFFIC_KEY = os.path.join(ROOT, "profiles", "gather_attn_kernel.json")
+
+
+def attention_traffic(rows: int, key_path: str = None):
+    """DRAM bytes of one gather_attn_kernel launch from the committed ncu
+    counters (profiles/gather_attn_kernel.json: bytes per query block, scaled
+    by the launch's query blocks -- the kernel's DRAM traffic is its
+    compulsory Q/K/V/O bytes, which grow with the query blocks).  None when
+    the kernel source differs from the one the counters were taken on:
+    attention.cu, common.cuh and the gather-attention part of kernels.cuh
+    (from its "---- gather attention" heading on)."""
     import hashlib
-    import re
     csrc = os.path.join(ROOT, "block_sparse_attention_20_b200", "csrc")
     try:
         src = attention_source(csrc)
-        txt = open(os.path.join(ROOT, "profiles", "gather_attn_kernel_wan1.3b.md")).read()
-    except OSError:
+        with open(key_path or TRAFFIC_KEY) as f:
+            key = json.load(f)
+    except (OSError, ValueError):
         return None
-    m = re.search(r"source sha256 ([0-9a-f]{16}); DRAM bytes per query block: ([0-9]+)", txt)
-    if not m or m.group(1) != hashlib.sha256(src).hexdigest()[:16]:
+    if key.get("source_sha256_16") != hashlib.sha256(src).hexdigest()[:16]:
         return None
-    return int(m.group(2)) * rows
+    return int(key["dram_bytes_per_query_block"]) * rows
 
 
 def run_sweep(args):
@@ -236,13 +244,31 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def bench_config(w, args) -> dict:
+    """The workload description both arms print (same keys, same values)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters,
+            "kmeans_iters": w.iters, "selection": args.selection,
+            "scoring": args.scoring, "draws": args.draws,
+            "per_rank": ("heads [r*H/N, (r+1)*H/N) of one problem" if args.split == "heads"
+                         else "one batch element per GPU"),
+            "l2": "inputs (Q,K,V 2.3 GB) exceed the 126 MB L2; no flush"}
+
+
 def run_reference(args, w):
     """The tier's reference arm: the float64 CPU oracle, as it stands, on a
-    bounded sample of query blocks per step."""
+    bounded sample of query blocks per step (every k-th row).  `value` is the
+    dense-equivalent throughput of the whole workload at the measured rate
+    (the measured time per sampled row times the workload's rows); the timed
+    region itself is `ms_per_step` x `steps`."""
     import oracle
 
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
+        return
+    if args.selection != "sip" or args.scoring != "keys" or args.draws != "independent":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the oracle's forward pass covers the method's own sampler and scoring only"}))
         return
     cores = oracle.default_threads()
     Q, K, V = synth.generate(w)
@@ -259,18 +285,21 @@ def run_reference(args, w):
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
-    dt = (time.perf_counter() - t0) / args.steps
-    full = dt * w.rows / len(rows)  # extrapolated to the whole workload
+    dt = (time.perf_counter() - t0) / args.steps  # measured seconds per step (the sample)
+    scale = w.rows / len(rows)
+    full = dt * scale  # the whole workload at the measured rate
     dense = 4.0 * w.B * w.H * w.N * w.N * w.d
     value = dense / full / 1e12
-    sample = f"{len(rows)} of {w.rows} query blocks per step (every {stride}th), time x{w.rows / len(rows):.1f}"
+    sample = (f"{len(rows)} of {w.rows} query blocks per step (every {stride}th); value scales the "
+              f"measured time x{scale:.1f} to the whole workload")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS (dense-equivalent)",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": full * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters},
+        "config": bench_config(w, args),
+        "extrapolated_ms_per_workload": full * 1e3,
+        "rows_per_step": int(len(rows)),
         "cpu_baseline": {"value": value, "unit": "TFLOPS (dense-equivalent)", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS (dense-equivalent)", "h2d_bytes_per_step": 0,
@@ -279,8 +308,10 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, Q, K, V, budget_s=15.0):
-    """The oracle on this host's cores, on a bounded sample of the workload."""
+def cpu_baseline(w, Q, K, V):
+    """The oracle on this host's cores, on a bounded sample of the workload:
+    the whole path (k-means, block probabilities, draw, weighted attention)
+    and, separately, dense float64 attention on the same query blocks."""
     import oracle
 
     cores = oracle.default_threads()
@@ -293,6 +324,12 @@ def cpu_baseline(w, Q, K, V, budget_s=15.0):
     dt = time.perf_counter() - t0
     full = dt * w.rows / len(rows)
     dense = 4.0 * w.B * w.H * w.N * w.N * w.d
+    # dense attention (O1) on a quarter of the same rows
+    drows = rows[::4]
+    t0 = time.perf_counter()
+    oracle.dense_attention(Q, K, V, w.shape, drows, nthreads=cores)
+    dt_dense = time.perf_counter() - t0
+    full_dense = dt_dense * w.rows / len(drows)
     # and the whole tiny workload (every query block) on one thread
     tw = synth.TINY
     Qt, Kt, Vt = synth.generate(tw)
@@ -304,17 +341,38 @@ def cpu_baseline(w, Q, K, V, budget_s=15.0):
             "kind": "oracle",
             "sample": f"{len(rows)} of {w.rows} query blocks (every {stride}th), {dt:.1f} s, "
                       f"extrapolated x{w.rows / len(rows):.1f}",
+            "dense_attention": {"value": dense / full_dense / 1e12, "unit": "TFLOPS",
+                                "sample": f"{len(drows)} query blocks, {dt_dense:.1f} s, "
+                                          f"extrapolated x{w.rows / len(drows):.1f}",
+                                "extrapolated_s": full_dense},
             "tiny_one_thread_s": dt1}
 
 
-def rank_plan(w, rank: int, world: int) -> dict:
-    """What rank `rank` of `world` computes (weak scaling, no collective on the
-    data path): batch elements [rank*B, (rank+1)*B) of a world*B-element
-    problem.  Its inputs are drawn with data seed w.seed + rank; its sampler
-    uses the global batch index (batch_offset) with the job's one Philox key."""
+def rank_plan(w, rank: int, world: int, split: str = "batch") -> dict:
+    """What rank `rank` of `world` computes; no collective on the data path.
+
+    split="batch" (weak scaling): batch elements [rank*B, (rank+1)*B) of a
+    world*B-element problem, inputs drawn with data seed w.seed + rank, the
+    sampler on the global batch index (batch_offset) with the job's one
+    Philox key.
+    split="heads" (strong scaling): heads [rank*H//world, (rank+1)*H//world)
+    of the one problem (data seed w.seed), the sampler on the global head
+    index (head_offset), so the job draws exactly what one call over all
+    heads draws."""
     if not 0 <= rank < world:
         raise ValueError(f"rank {rank} outside world {world}")
-    return {"batch_offset": rank * w.B, "data_seed": w.seed + rank, "philox_seed": w.seed}
+    if split == "batch":
+        return {"batch_offset": rank * w.B, "head_offset": 0, "heads": w.H, "data_seed": w.seed + rank,
+                "philox_seed": w.seed}
+    if split == "heads":
+        if world > w.B * w.H:
+            raise ValueError(f"{world} ranks for {w.B * w.H} heads")
+        if w.B != 1:
+            raise ValueError("the head split shares out the heads of one batch element")
+        h0, h1 = rank * w.H // world, (rank + 1) * w.H // world
+        return {"batch_offset": 0, "head_offset": h0, "heads": h1 - h0, "data_seed": w.seed,
+                "philox_seed": w.seed}
+    raise ValueError(f"unknown split {split!r}")
 
 
 def max_over_ranks(x: float, world: int, device=None) -> float:
@@ -332,6 +390,28 @@ def job_value(flop_per_rank: float, world: int, ms: float) -> float:
     """Whole-job dense-equivalent TFLOPS: the work of all ranks over the
     slowest rank's time."""
     return flop_per_rank * world / (ms * 1e-3) / 1e12
+
+
+def rank_inputs(w, plan):
+    """This rank's Q, K, V (CPU bf16) and its share of the workload."""
+    if plan["heads"] == w.H and plan["head_offset"] == 0:
+        return synth.generate(w.with_(seed=plan["data_seed"])), w
+    Q, K, V = synth.generate(w.with_(seed=plan["data_seed"]))
+    h0, h1 = plan["head_offset"], plan["head_offset"] + plan["heads"]
+    return tuple(t[:, h0:h1].contiguous() for t in (Q, K, V)), w.with_(H=h1 - h0)
+
+
+def roofline_peaks(pk: dict, sm_mhz):
+    """(burst peak, peak scaled to the sampled SM clock) in TFLOP/s.
+
+    The burst figure is cuBLAS bf16 timed alone; the sustained figure was
+    measured at the median clock recorded beside it, so scaling it by the
+    clock this run saw gives the peak at this run's clock."""
+    burst = float(pk.get("bf16_tflops", FALLBACK_PEAK_TFLOPS))
+    sus = pk.get("bf16_tflops_sustained")
+    mhz = (pk.get("clocks_under_load") or {}).get("sm_mhz_median")
+    scaled = float(sus) * float(sm_mhz) / float(mhz) if sus and mhz and sm_mhz else None
+    return burst, scaled
 
 
 def main():
@@ -360,18 +440,18 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    plan = rank_plan(w, rank, world)
-    Qc, Kc, Vc = synth.generate(w.with_(seed=plan["data_seed"]))
+    plan = rank_plan(w, rank, world, args.split)
+    (Qc, Kc, Vc), wr = rank_inputs(w, plan)
     Q, K, V = Qc.to(dev), Kc.to(dev), Vc.to(dev)
-    shape = w.shape
+    shape = wr.shape
     cfg = abatt.Config(kv_block=w.Bk, clusters=w.clusters, kmeans_iters=w.iters,
                        budget_bp=w.budget_bp, seed=plan["philox_seed"],
-                       batch_offset=plan["batch_offset"],
+                       batch_offset=plan["batch_offset"], head_offset=plan["head_offset"],
                        selection=abatt.SELECT_TOPK if args.selection == "topk" else abatt.SELECT_SIP,
                        scoring=(abatt.SCORE_BLOCK_MEANS if args.scoring == "block-means"
                                 else abatt.SCORE_KEYS),
                        draws=abatt.DRAWS_PAIRED if args.draws == "paired" else abatt.DRAWS_INDEPENDENT)
-    rows, nK = w.rows, w.nK
+    rows, nK = wr.rows, wr.nK
     p = torch.empty((rows, nK), dtype=torch.float32, device=dev)
     counts = torch.empty(rows, dtype=torch.int32, device=dev)
     idx = torch.empty((rows, nK), dtype=torch.int32, device=dev)
@@ -384,7 +464,8 @@ def main():
                          device=dev)
     stream = torch.cuda.current_stream()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # events: select | sample | pair segments | gather attention
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
 
     def step(e=None):
         if e: e[0].record(stream)
@@ -392,8 +473,10 @@ def main():
         if e: e[1].record(stream)
         abatt.sample(p, shape, cfg, out=(counts, idx, logw), workspace=ws_small, stream=stream)
         if e: e[2].record(stream)
-        abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws_att, stream=stream)
+        abatt.attention_plan(shape, counts, idx, logw, cfg, workspace=ws_att, stream=stream)
         if e: e[3].record(stream)
+        abatt.attention_planned(Q, K, V, cfg, workspace=ws_att, out=O, stream=stream)
+        if e: e[4].record(stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -414,10 +497,10 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
-    sel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
-    smp_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
-    att_ms = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
-    att_mean = sum(e[2].elapsed_time(e[3]) for e in ev) / len(ev)
+    med = lambda a, b: statistics.median(e[a].elapsed_time(e[b]) for e in ev)
+    sel_ms, smp_ms, plan_ms, gat_ms = med(0, 1), med(1, 2), med(2, 3), med(3, 4)
+    att_ms = med(2, 4)
+    gat_mean = sum(e[3].elapsed_time(e[4]) for e in ev) / len(ev)
     ms_step = total_ms / args.steps
     status = abatt.read_status(ws_small) | abatt.read_status(ws_sel) | abatt.read_status(ws_att)
 
@@ -426,28 +509,30 @@ def main():
     bpt = 128 // w.Bk
     # executed tiles: every row runs its own drawn blocks, 128/Bk per tile
     # (pairs of neighbouring rows share the gathers of common tiles, not the math)
-    last = w.nK - 1
-    tail = w.N - last * w.Bk
+    last = wr.nK - 1
+    tail = wr.N - last * wr.Bk
     keys = np.zeros(rows, dtype=np.int64)
     for r in range(rows):
         L = c[r]
-        keys[r] = L * w.Bk - (w.Bk - tail if L and idx_h[r, :L][-1] == last else 0)
+        keys[r] = L * wr.Bk - (wr.Bk - tail if L and idx_h[r, :L][-1] == last else 0)
     tiles = int(((c + bpt - 1) // bpt).sum())
-    exec_flop = tiles * 4.0 * 128 * 128 * w.d
+    exec_flop = tiles * 4.0 * 128 * 128 * wr.d
     # algorithmic work: valid query rows x valid drawn keys
-    nrows_q = np.minimum(128, w.N - (np.arange(rows) % w.nQ) * 128)
-    alg_flop = float((4.0 * w.d * nrows_q * keys).sum())
-    dense_flop = 4.0 * w.B * w.H * w.N * w.N * w.d
-    skip = 1.0 - float((nrows_q * keys).sum()) / (w.B * w.H * w.N * float(w.N))
+    nrows_q = np.minimum(128, wr.N - (np.arange(rows) % wr.nQ) * 128)
+    alg_flop = float((4.0 * wr.d * nrows_q * keys).sum())
+    rank_dense = 4.0 * wr.B * wr.H * wr.N * wr.N * wr.d
+    job_dense = 4.0 * w.B * w.H * w.N * w.N * w.d * (world if args.split == "batch" else 1)
+    skip = 1.0 - float((nrows_q * keys).sum()) / (wr.B * wr.H * wr.N * float(wr.N))
 
     pk, src = peaks()
-    peak = float(pk.get("bf16_tflops_sustained") or pk["bf16_tflops"])
-    achieved = alg_flop / (att_mean * 1e-3) / 1e12
+    clocks = clk.summary()
+    burst, at_clock = roofline_peaks(pk, clocks.get("sm_mhz"))
+    achieved = alg_flop / (gat_mean * 1e-3) / 1e12
     # blocks the two rows of a pair both drew (gathered once for both), over
     # the blocks either drew
     both = either = 0
     for r in range(0, rows - 1, 2):
-        if (r % w.nQ) % 2 or r // w.nQ != (r + 1) // w.nQ:
+        if (r % wr.nQ) % 2 or r // wr.nQ != (r + 1) // wr.nQ:
             continue
         a0, a1 = idx_h[r, :c[r]], idx_h[r + 1, :c[r + 1]]
         k = np.intersect1d(a0, a1, assume_unique=True).size
@@ -456,37 +541,38 @@ def main():
 
     line = {
         "metric": METRIC,
-        "value": job_value(dense_flop, world, ms_step),
+        "value": job_value(job_dense, 1, ms_step),
         "unit": "TFLOPS (dense-equivalent)",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak" if args.split == "batch" else "strong",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "budget_bp": w.budget_bp, "kv_block": w.Bk, "clusters": w.clusters,
-                   "kmeans_iters": w.iters, "selection": args.selection,
-                   "scoring": args.scoring, "draws": args.draws,
-                   "per_rank": "one batch element per GPU",
-                   "l2": "inputs (Q,K,V 2.3 GB) exceed the 126 MB L2; no flush"},
-        "stages_ms": {"select": sel_ms, "sample": smp_ms, "attention": att_ms},
+        "config": bench_config(w, args),
+        "stages_ms": {"select": sel_ms, "sample": smp_ms, "attention": att_ms,
+                      "attention_pair_segments": plan_ms, "attention_gather_kernel": gat_ms},
         "attention_ms": att_ms,
         "selector_sampler_share": (sel_ms + smp_ms) / (sel_ms + smp_ms + att_ms),
         "realized_skip": skip,
         "pair_shared_fraction": both / max(either, 1),
-        "executed_tflops_attention": exec_flop / (att_mean * 1e-3) / 1e12,
+        "executed_tflops_attention": exec_flop / (gat_mean * 1e-3) / 1e12,
         "algorithmic_tflops_attention": achieved,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": attention_traffic(rows),
-                     "kernel": "gather_attn_kernel", "flops": "algorithmic (valid query rows x drawn keys)",
-                     "peak_source": f"{src} bf16 sustained"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                     "frac": achieved / burst, "traffic": attention_traffic(rows),
+                     "kernel": "gather_attn_kernel (timed alone, CUDA events on its stream)",
+                     "flops": "algorithmic (valid query rows x drawn keys)",
+                     "peak_source": f"{src} bf16 burst",
+                     "peak_at_sampled_clock": at_clock,
+                     "frac_at_sampled_clock": achieved / at_clock if at_clock else None},
+        "rank_dense_tflop": rank_dense / 1e12,
         "device_status": status,
         "gpu_launches": 7 * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
 
     if not args.no_keep_all:
-        line["keep_all"] = keep_all(abatt, cfg, Q, K, V, w, O, ws_att, stream)
+        line["keep_all"] = keep_all(abatt, cfg, Q, K, V, wr, O, ws_att, stream)
     if not args.no_e2e:
-        line["e2e"] = e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world)
+        line["e2e"] = e2e(abatt, cfg, Qc, Kc, Vc, dev, wr, args, world, job_dense)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the host baseline: one process alone
         line["cpu_baseline"] = cpu_baseline(w, Qc, Kc, Vc)
     if rank == 0:
@@ -498,36 +584,39 @@ def main():
 
 def keep_all(abatt, cfg, Q, K, V, w, O, ws, stream):
     """The same attention kernel fed every key block with weight 1 (dense
-    attention through the gather path), timed the same way."""
+    attention through the gather path), timed the same way: the pair
+    segments once, then the gather kernel alone."""
     import torch
 
     rows, nK = w.rows, w.nK
     counts = torch.full((rows,), nK, dtype=torch.int32, device=Q.device)
     idx = torch.arange(nK, dtype=torch.int32, device=Q.device).repeat(rows, 1)
     logw = torch.zeros((rows, nK), dtype=torch.float32, device=Q.device)
+    abatt.attention_plan(w.shape, counts, idx, logw, cfg, workspace=ws, stream=stream)
     for _ in range(2):
-        abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws, stream=stream)
+        abatt.attention_planned(Q, K, V, cfg, workspace=ws, out=O, stream=stream)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     reps = 3
     a.record(stream)
     for _ in range(reps):
-        abatt.attention(Q, K, V, counts, idx, logw, cfg, out=O, workspace=ws, stream=stream)
+        abatt.attention_planned(Q, K, V, cfg, workspace=ws, out=O, stream=stream)
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     dense = 4.0 * w.B * w.H * w.N * w.N * w.d
     tiles = rows * ((nK + 128 // w.Bk - 1) // (128 // w.Bk))
-    return {"attention_ms": ms, "dense_tflops": dense / (ms * 1e-3) / 1e12,
+    return {"gather_kernel_ms": ms, "dense_tflops": dense / (ms * 1e-3) / 1e12,
             "executed_tflops": tiles * 4.0 * 128 * 128 * w.d / (ms * 1e-3) / 1e12}
 
 
-def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):
+def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world, job_dense):
     """Same metric through the public host-to-host call: every step copies
     Q, K, V from pinned host memory to the device and O back, through
     abatt.HostPipeline (abatt_forward over chunks of heads, the copies of one
-    chunk overlapped with the compute of the previous one)."""
+    chunk overlapped with the compute of the previous one).  `w` is this
+    rank's share; `job_dense` the whole job's dense-equivalent FLOPs."""
     import torch
     import torch.distributed as dist
 
@@ -553,9 +642,8 @@ def e2e(abatt, cfg, Qc, Kc, Vc, dev, w, args, world):
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
-    dense = 4.0 * w.B * w.H * w.N * w.N * w.d
     nbytes = Qc.numel() * 2
-    return {"value": job_value(dense, world, ms), "unit": "TFLOPS (dense-equivalent)",
+    return {"value": job_value(job_dense, 1, ms), "unit": "TFLOPS (dense-equivalent)",
             "ms_per_step": ms, "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
             "steps": steps, "heads_per_chunk": pipe.hc, "device_status": pipe.status()}
 

@@ -25,12 +25,16 @@ SCORE_KEYS, SCORE_BLOCK_MEANS = 0, 1
 LAYOUT_BHND, LAYOUT_BNHD = 0, 1
 DRAWS_INDEPENDENT, DRAWS_PAIRED = 0, 1
 DEVFLAG_CAPACITY, DEVFLAG_TIMEOUT, DEVFLAG_BADLIST = 0x1, 0x2, 0x4
+NOALLOC_STATUS_PENDING = 0xFFFFFFFF
+TEST_WAIT_NS, TEST_STALL = 1, 2
+TEST_STALL_ATTENTION, TEST_STALL_SCORE = 0x1, 0x2
 
 # Every symbol declared in include/abatt.h.
 EXPORTS = (
     "abatt_workspace_size", "abatt_select", "abatt_sample", "abatt_attention", "abatt_forward",
     "abatt_forward_intermediates", "abatt_read_status", "abatt_clear_status",
     "abatt_status_string", "abatt_version", "abatt_attention_noalloc",
+    "abatt_attention_plan", "abatt_attention_planned", "abatt_test_set", "abatt_test_exp2_poly",
 )
 
 
@@ -101,6 +105,10 @@ def lib():
         L.abatt_attention.argtypes = [P, P, P, S, C, P, P, P, i32, P, P, P, sz, P]
         L.abatt_forward.argtypes = [P, P, P, S, C, P, P, P, sz, P]
         L.abatt_attention_noalloc.argtypes = [P, P, P, S, C, P, P, P, i32, P, P, P, P]
+        L.abatt_attention_plan.argtypes = [S, C, P, P, P, i32, P, sz, P]
+        L.abatt_attention_planned.argtypes = [P, P, P, S, C, P, P, P, sz, P]
+        L.abatt_test_set.argtypes = [i32, ctypes.c_uint64]
+        L.abatt_test_exp2_poly.argtypes = [P, P, ctypes.c_int64, i32, P]
         L.abatt_forward_intermediates.argtypes = [P, S, C, ctypes.POINTER(P), ctypes.POINTER(P),
                                                   ctypes.POINTER(P), ctypes.POINTER(P)]
         L.abatt_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
@@ -162,6 +170,48 @@ def _check_bf16(*ts):
                              "[B, N, H, d] with layout=LAYOUT_BNHD)")
 
 
+def _check_qkv(q, k, v=None):
+    """Q, K (and V): contiguous CUDA bf16 4-D tensors of one shape on one device."""
+    ts = (q, k) if v is None else (q, k, v)
+    _check_bf16(*ts)
+    if q.dim() != 4:
+        raise ValueError(f"Q must be 4-D, got shape {tuple(q.shape)}")
+    for name, t in zip("KV", ts[1:]):
+        if t.shape != q.shape or t.device != q.device:
+            raise ValueError(f"{name} must have Q's shape {tuple(q.shape)} and device {q.device}, "
+                             f"got {tuple(t.shape)} on {t.device}")
+
+
+def _check_tensor(t, name, dtype, shape, device):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch tensor")
+    if t.dtype != dtype or t.device != device or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on {device}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _check_lists(counts, idx, logw, rows, device):
+    """counts int32 [rows]; idx int32 and logw fp32 [rows, capacity] (capacity >= 1)."""
+    import torch
+    if idx.dim() != 2 or idx.shape[1] < 1:
+        raise ValueError(f"idx must be [rows, capacity] with capacity >= 1, got {tuple(idx.shape)}")
+    cap = idx.shape[1]
+    _check_tensor(counts, "counts", torch.int32, (rows,), device)
+    _check_tensor(idx, "idx", torch.int32, (rows, cap), device)
+    _check_tensor(logw, "logw", torch.float32, (rows, cap), device)
+    return cap
+
+
+def _check_outputs(q, out, lse, sh):
+    import torch
+    if out is not None:
+        _check_tensor(out, "out", torch.bfloat16, q.shape, q.device)
+    if lse is not None:
+        _check_tensor(lse, "lse", torch.float32, (sh.B, sh.H, sh.N), q.device)
+
+
 def workspace_size(call: int, shape, cfg: Config) -> int:
     sh = shape if isinstance(shape, _Shape) else _Shape(*shape)
     out = ctypes.c_size_t()
@@ -186,7 +236,7 @@ def select(q, k, cfg: Config, *, p=None, want_centroids=False, workspace=None, s
     With ``want_centroids`` also returns the fp32 centroids [rows, C, d] and
     cluster sizes [rows, C]."""
     import torch
-    _check_bf16(q, k)
+    _check_qkv(q, k)
     sh = _shape_of(q, cfg)
     nQ, nK, rows = _geom(sh, cfg)
     if p is None:
@@ -227,12 +277,13 @@ def attention(q, k, v, counts, idx, logw, cfg: Config, *, out=None, want_lse=Fal
               workspace=None, stream=None):
     """Gather attention over the listed blocks.  Returns O (and lse)."""
     import torch
-    _check_bf16(q, k, v)
+    _check_qkv(q, k, v)
     sh = _shape_of(q, cfg)
-    cap = idx.shape[1]
+    cap = _check_lists(counts, idx, logw, _geom(sh, cfg)[2], q.device)
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((sh.B, sh.H, sh.N), dtype=torch.float32, device=q.device) if want_lse else None
+    _check_outputs(q, out, lse, sh)
     ws = _workspace(CALL_ATTENTION, sh, cfg, q.device, workspace)
     _check(lib().abatt_attention(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(sh),
                                  ctypes.byref(cfg._c(sh.d)), _ptr(counts), _ptr(idx), _ptr(logw),
@@ -251,26 +302,82 @@ def attention_noalloc(q, k, v, counts, idx, logw, cfg: Config, *, out, lse=None,
     For callers that cannot allocate device memory: its scratch is a fixed
     64 MiB array inside the library, shared by every call on a device (calls
     that overlap on the GPU race on it).  The caller supplies every input and
-    output buffer, including `out` (and `lse`, `dev_status` if wanted)."""
-    _check_bf16(q, k, v)
+    output buffer, including `out` (and `lse`, `dev_status` if wanted); this
+    wrapper checks their shapes, dtypes and devices and allocates nothing."""
+    import torch
+    _check_qkv(q, k, v)
     sh = _shape_of(q, cfg)
+    cap = _check_lists(counts, idx, logw, _geom(sh, cfg)[2], q.device)
+    if out is None:
+        raise ValueError("out is required (the call allocates nothing)")
+    _check_outputs(q, out, lse, sh)
+    if dev_status is not None:
+        if dev_status.dtype not in (torch.int32, torch.uint32) or dev_status.numel() != 1 \
+                or dev_status.device != q.device:
+            raise ValueError("dev_status must be a one-element int32 or uint32 tensor on Q's device")
     _check(lib().abatt_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(sh),
                                          ctypes.byref(cfg._c(sh.d)), _ptr(counts), _ptr(idx),
-                                         _ptr(logw), idx.shape[1], _ptr(out), _ptr(lse),
+                                         _ptr(logw), cap, _ptr(out), _ptr(lse),
                                          _ptr(dev_status), _stream(stream)),
            "abatt_attention_noalloc")
     return out
+
+
+def attention_plan(shape, counts, idx, logw, cfg: Config, *, workspace, stream=None):
+    """First launch of :func:`attention`: the pair segments, into `workspace`
+    (an ATTENTION workspace; its status word is cleared)."""
+    sh = shape if isinstance(shape, _Shape) else _Shape(*shape)
+    cap = _check_lists(counts, idx, logw, _geom(sh, cfg)[2], counts.device)
+    ws = _workspace(CALL_ATTENTION, sh, cfg, counts.device, workspace)
+    _check(lib().abatt_attention_plan(ctypes.byref(sh), ctypes.byref(cfg._c(sh.d)), _ptr(counts), _ptr(idx),
+                                      _ptr(logw), cap, _ptr(ws), ws.numel(), _stream(stream)),
+           "abatt_attention_plan")
+    return ws
+
+
+def attention_planned(q, k, v, cfg: Config, *, workspace, out=None, want_lse=False, stream=None):
+    """Second launch of :func:`attention`: the gather-attention kernel on the
+    plan that :func:`attention_plan` left in `workspace`."""
+    import torch
+    _check_qkv(q, k, v)
+    sh = _shape_of(q, cfg)
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((sh.B, sh.H, sh.N), dtype=torch.float32, device=q.device) if want_lse else None
+    _check_outputs(q, out, lse, sh)
+    ws = _workspace(CALL_ATTENTION, sh, cfg, q.device, workspace)
+    _check(lib().abatt_attention_planned(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(sh),
+                                         ctypes.byref(cfg._c(sh.d)), _ptr(out), _ptr(lse), _ptr(ws),
+                                         ws.numel(), _stream(stream)), "abatt_attention_planned")
+    return (out, lse) if want_lse else out
+
+
+def test_set(hook: int, value: int) -> None:
+    """Test hook of the library (TEST_WAIT_NS, TEST_STALL; see abatt_test_set)."""
+    _check(lib().abatt_test_set(int(hook), int(value) & (2**64 - 1)), "abatt_test_set")
+
+
+def test_exp2_poly(x, degree: int, stream=None):
+    """2^x (fp32 CUDA tensor) through the kernels' FMA-pipe polynomial."""
+    import torch
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    _check(lib().abatt_test_exp2_poly(_ptr(x), _ptr(y), x.numel(), int(degree), _stream(stream)),
+           "abatt_test_exp2_poly")
+    return y
 
 
 def forward(q, k, v, cfg: Config, *, out=None, want_lse=False, workspace=None, stream=None):
     """The whole path.  Returns O (and lse); pass ``workspace`` to keep the
     intermediates (see :func:`intermediates`)."""
     import torch
-    _check_bf16(q, k, v)
+    _check_qkv(q, k, v)
     sh = _shape_of(q, cfg)
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((sh.B, sh.H, sh.N), dtype=torch.float32, device=q.device) if want_lse else None
+    _check_outputs(q, out, lse, sh)
     ws = _workspace(CALL_FORWARD, sh, cfg, q.device, workspace)
     _check(lib().abatt_forward(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(sh),
                                ctypes.byref(cfg._c(sh.d)), _ptr(out), _ptr(lse), _ptr(ws),

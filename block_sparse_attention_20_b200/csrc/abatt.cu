@@ -4,6 +4,7 @@
 // abatt_read_status.
 #include <math.h>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string.h>
 
@@ -14,6 +15,10 @@ using namespace abatt;
 namespace {
 
 constexpr uint64_t kWaitNs = 500000000ull;  // bounded waits give up after ~0.5 s
+
+// Test hooks (abatt_test_set): the bounded-wait limit and the producer stall.
+std::atomic<uint64_t> g_wait_ns{kWaitNs};
+std::atomic<uint32_t> g_stall{0};
 constexpr float kLog2eF = 1.4426950408889634f;
 
 struct Geom {
@@ -262,7 +267,8 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     sa.mref = at<float>(ws, L.mref);
     sa.mz = at<float2>(ws, L.mz);
     sa.hdr = at<WsHeader>(ws, L.hdr);
-    sa.wait_ns = kWaitNs;
+    sa.wait_ns = g_wait_ns.load();
+    sa.stall = (g_stall.load() & ABATT_TEST_STALL_SCORE) ? 1 : 0;
     sa.C = g.C;
     sa.weight = ka.weight;
     sa.p = p;
@@ -302,11 +308,8 @@ abatt_status run_sample(const float *p, const Geom &g, const abatt_config *cfg, 
     return cuda_status(launch_sample(a, sms, st));
 }
 
-abatt_status run_attention(const void *Q, const void *K, const void *V, const Geom &g,
-                           const abatt_config *cfg, const int32_t *counts, const int32_t *idx,
-                           const float *logw, int capacity, void *O, float *lse, void *ws,
-                           const Layout &L, int sms, cudaStream_t st) {
-    WsHeader *hdr = at<WsHeader>(ws, L.hdr);
+PairArgs pair_args(const Geom &g, const int32_t *counts, const int32_t *idx, const float *logw, int capacity,
+                   void *ws, const Layout &L) {
     PairArgs pa;
     pa.rows = g.rows; pa.pairs = pairs_of(g); pa.nQ = g.nQ; pa.nK = g.nK; pa.capacity = capacity; pa.cap_u = g.nK;
     pa.counts = counts; pa.idx = idx; pa.logw = logw;
@@ -316,9 +319,22 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     pa.useg = at<int32_t>(ws, L.useg);
     pa.ublk = at<int32_t>(ws, L.ublk);
     pa.ulw = at<float>(ws, L.ulw);
-    pa.status = &hdr->status;
-    if (launch_pair_union(pa, sms, st) != cudaSuccess) return ABATT_ERR_CUDA;
+    pa.status = &at<WsHeader>(ws, L.hdr)->status;
+    return pa;
+}
 
+// Pair segments of every pair of query blocks (the first launch of attention).
+abatt_status run_plan(const Geom &g, const int32_t *counts, const int32_t *idx, const float *logw,
+                      int capacity, void *ws, const Layout &L, int sms, cudaStream_t st) {
+    const PairArgs pa = pair_args(g, counts, idx, logw, capacity, ws, L);
+    return cuda_status(launch_pair_union(pa, sms, st));
+}
+
+// Gather attention from the pair segments in the workspace (the second launch).
+abatt_status run_planned(const void *Q, const void *K, const void *V, const Geom &g,
+                         const abatt_config *cfg, void *O, float *lse, void *ws, const Layout &L, int sms,
+                         cudaStream_t st) {
+    const PairArgs pa = pair_args(g, nullptr, nullptr, nullptr, 1, ws, L);
     const int CH = g.d / 64;
     const Strides sd = strides_of(g, cfg);
     const bool bnhd = cfg->layout == ABATT_LAYOUT_BNHD;
@@ -362,9 +378,19 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
     a.useg = pa.useg; a.ublk = pa.ublk; a.ulw = pa.ulw;
     a.O = static_cast<__nv_bfloat16 *>(O);
     a.lse = lse;
-    a.hdr = hdr;
-    a.wait_ns = kWaitNs;
+    a.hdr = at<WsHeader>(ws, L.hdr);
+    a.wait_ns = g_wait_ns.load();
+    a.stall = (g_stall.load() & ABATT_TEST_STALL_ATTENTION) ? 1 : 0;
     return cuda_status(launch_attention(a, m, sms, st));
+}
+
+abatt_status run_attention(const void *Q, const void *K, const void *V, const Geom &g,
+                           const abatt_config *cfg, const int32_t *counts, const int32_t *idx,
+                           const float *logw, int capacity, void *O, float *lse, void *ws,
+                           const Layout &L, int sms, cudaStream_t st) {
+    abatt_status s = run_plan(g, counts, idx, logw, capacity, ws, L, sms, st);
+    if (s != ABATT_OK) return s;
+    return run_planned(Q, K, V, g, cfg, O, lse, ws, L, sms, st);
 }
 
 // Scratch of abatt_attention_noalloc: status word and pair unions, in the
@@ -372,22 +398,74 @@ abatt_status run_attention(const void *Q, const void *K, const void *V, const Ge
 // name it directly; host code needs its address from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ABATT_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[64];
+// The address is only valid in the CUDA context it was looked up in (a reset
+// device or a context a host made with the driver API loads the module
+// again), so the cache is keyed on the current context's unique id.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current.
+template <typename F>
+F driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<F>(p);
+}
+
+// Unique id of the current context (0 and false when there is none).
+bool current_ctx_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+        get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    });
+    *id = 0;
+    CUcontext ctx = nullptr;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+struct ScratchEntry {
+    unsigned long long ctx_id;  // context the address belongs to
+    void *ptr;
+};
+std::mutex g_noalloc_mu;
+ScratchEntry g_noalloc[64];  // per device: the last context seen there
+
+// Device address of the scratch array in the current context, looked up with
+// cudaGetSymbolAddress the first time a context calls.
 abatt_status noalloc_scratch(void **ptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ABATT_ERR_CUDA;
+    unsigned long long id = 0;
+    const bool have_ctx = current_ctx_id(&id);
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!have_ctx || g_noalloc[dev].ctx_id != id || !g_noalloc[dev].ptr) {
+        // with no context current, this makes the device's primary context current
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ABATT_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        if (!current_ctx_id(&id)) return ABATT_ERR_CUDA;
+        g_noalloc[dev].ctx_id = id;
+        g_noalloc[dev].ptr = p;
     }
-    *ptr = g_noalloc_ptr[dev];
+    *ptr = g_noalloc[dev].ptr;
     return ABATT_OK;
+}
+
+// 2^x through the FMA-pipe polynomial of the kernels (test hook).
+template <int DEG>
+__global__ void exp2_poly_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t n) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x * 2;
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 2; i < n; i += stride) {
+        const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.0f);
+        const float2 r = exp2_poly2<DEG>(v);
+        y[i] = r.x;
+        if (i + 1 < n) y[i + 1] = r.y;
+    }
 }
 
 }  // namespace
@@ -478,6 +556,39 @@ abatt_status abatt_attention(const void *Q, const void *K, const void *V,
                          st);
 }
 
+abatt_status abatt_attention_plan(const abatt_shape *shape, const abatt_config *cfg,
+                                  const int32_t *counts, const int32_t *idx, const float *logw,
+                                  int capacity, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!counts || !idx || !logw || capacity < 1) return ABATT_ERR_INVALID_ARG;
+    if ((s = check_ws(ABATT_CALL_ATTENTION, g, workspace, workspace_bytes)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const Layout L = layout(ABATT_CALL_ATTENTION, g);
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
+    return run_plan(g, counts, idx, logw, capacity, workspace, L, sms, st);
+}
+
+abatt_status abatt_attention_planned(const void *Q, const void *K, const void *V,
+                                     const abatt_shape *shape, const abatt_config *cfg, void *O,
+                                     float *lse, void *workspace, size_t workspace_bytes,
+                                     void *stream) {
+    Geom g;
+    abatt_status s = validate(shape, cfg, &g);
+    if (s != ABATT_OK) return s;
+    if (!Q || !K || !V || !O) return ABATT_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return ABATT_ERR_ALIGNMENT;
+    if ((s = check_ws(ABATT_CALL_ATTENTION, g, workspace, workspace_bytes)) != ABATT_OK) return s;
+    int sms = 0;
+    if ((s = device_sms(&sms)) != ABATT_OK) return s;
+    const Layout L = layout(ABATT_CALL_ATTENTION, g);
+    return run_planned(Q, K, V, g, cfg, O, lse, workspace, L, sms, static_cast<cudaStream_t>(stream));
+}
+
 abatt_status abatt_attention_noalloc(const void *Q, const void *K, const void *V,
                                      const abatt_shape *shape, const abatt_config *cfg,
                                      const int32_t *counts, const int32_t *idx, const float *logw,
@@ -497,6 +608,9 @@ abatt_status abatt_attention_noalloc(const void *Q, const void *K, const void *V
     int sms = 0;
     if ((s = device_sms(&sms)) != ABATT_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // until this call's flags are copied there, dev_status reads "pending"
+    if (dev_status && cudaMemsetAsync(dev_status, 0xFF, sizeof(uint32_t), st) != cudaSuccess)
+        return ABATT_ERR_CUDA;
     // the status word must start at zero; the union lists are fully rewritten
     if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), st) != cudaSuccess) return ABATT_ERR_CUDA;
     s = run_attention(Q, K, V, g, cfg, counts, idx, logw, capacity, O, lse, scratch, L, sms, st);
@@ -546,6 +660,28 @@ abatt_status abatt_forward_intermediates(void *workspace, const abatt_shape *sha
     if (idx) *idx = at<int32_t>(workspace, L.idx);
     if (logw) *logw = at<float>(workspace, L.logw);
     return ABATT_OK;
+}
+
+abatt_status abatt_test_set(int hook, uint64_t value) {
+    switch (hook) {
+        case ABATT_TEST_WAIT_NS: g_wait_ns.store(value ? value : kWaitNs); return ABATT_OK;
+        case ABATT_TEST_STALL: g_stall.store((uint32_t)value); return ABATT_OK;
+    }
+    return ABATT_ERR_INVALID_ARG;
+}
+
+abatt_status abatt_test_exp2_poly(const float *x, float *y, int64_t n, int degree, void *stream) {
+    if (!x || !y || n < 0 || (degree != 3 && degree != 4)) return ABATT_ERR_INVALID_ARG;
+    if (n == 0) return ABATT_OK;
+    int sms = 0;
+    abatt_status s = device_sms(&sms);
+    if (s != ABATT_OK) return s;
+    int64_t grid = (n + 511) / 512;
+    if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (degree == 3) exp2_poly_kernel<3><<<(unsigned)grid, 256, 0, st>>>(x, y, n);
+    else exp2_poly_kernel<4><<<(unsigned)grid, 256, 0, st>>>(x, y, n);
+    return cuda_status(cudaGetLastError());
 }
 
 abatt_status abatt_read_status(const void *workspace, uint32_t *flags, void *stream) {

@@ -4,20 +4,27 @@
 // sentence: each drawn block is re-weighted by 1/pi, here as +ln(1/pi) on
 // its logits inside the online softmax).
 //
-// B200 design.  On this GPU the kernel is bound by how fast gathered K/V
-// bytes move from L2 to the SMs, not by the tensor cores, so neighbouring
-// query blocks share their gathers:
+// B200 design.  Neighbouring query blocks (rows 2p and 2p+1 of a head, a
+// "pair") draw heavily overlapping lists, so they run together on one SM and
+// share the gathers of the blocks both drew:
 //
-//   pair_union_kernel   rows 2p and 2p+1 (a "pair") get one ascending union
-//                       of their two drawn lists, with each row's log-weight
-//                       per union block (-1 where the row did not draw it).
+//   pair_union_kernel   lays the pair's two ascending lists out as one array
+//                       of three ascending segments, [blocks both rows drew |
+//                       row 0 only | row 1 only], with each row's base-2
+//                       log-weights in the order that row walks them
+//                       ([both | its own]; -inf up to the end of its last
+//                       tile) and the position of the partial last key block.
 //   gather_attn_kernel  persistent, one CTA per SM, one pair at a time.  Each
-//                       128-key tile of the union is gathered once (one 4 KB
-//                       TMA box per 16-key block for K and for V) and used by
-//                       both rows; a row gives the blocks it did not draw a
-//                       -inf logit, so they add exactly zero.
+//                       row walks exactly its own blocks in 128-key tiles, so
+//                       no tile holds a block the row did not draw; tiles that
+//                       lie wholly inside the shared segment are gathered once
+//                       (TMA boxes of one key block each, K and V) for both
+//                       rows, later tiles per row.
 //
-//   tensor core, per tile t:   S0(t)  PV1(t-1)  S1(t)  PV0(t)
+// What bounds it is the per-row chain S(t) -> softmax(t) -> PV(t) -> S(t+1)
+// (P replaces S in tensor memory): the softmax of a 128x128 tile is bound by
+// issue slots and the ex2 unit, and the two rows' softmaxes overlap the other
+// row's tensor-core work only partly.
 //
 // Warp roles (640 threads, five warpgroups; warpgroup 0 hands registers to
 // the softmax warpgroups with setmaxnreg):
@@ -34,9 +41,6 @@
 //               shuffle, lazy running maximum (O is rescaled only when it
 //               grows by more than 8), P in bf16 back into tensor memory,
 //               final O / l to bf16 (each thread writes half of its row).
-//               The softmax latency of a tile sits on each row's critical
-//               path (P replaces S in tensor memory, so S(t+1) waits for
-//               PV(t)); two threads per row halve it.
 #include "kernels.cuh"
 
 namespace abatt {
@@ -262,9 +266,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
 
+    __shared__ int skip_s;
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT))
-        return;  // a bounded wait elsewhere already gave up: start no more work
+    // a bounded wait elsewhere already gave up: start no more work.  One read,
+    // shared by the whole CTA, so every role takes the same decision
+    if (threadIdx.x == 0)
+        skip_s = a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT);
+    __syncthreads();
+    if (skip_s) return;
     const WaitCtx wc{&abort_s, a.hdr, a.wait_ns};
 
     if (threadIdx.x == 0) {
@@ -293,7 +303,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
 
-    uint32_t ring_issued = 0;  // producer: ring loads issued (for the drain)
+    uint32_t ring_issued = 0;         // producer: ring loads issued (for the drain)
+    uint32_t q_issued[2] = {0, 0};    // producer: Q loads issued per row slot (for the drain)
 
     if (warp == 0) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
@@ -338,10 +349,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int c = 0; c < CH; ++c)
                         tma_load_4d(sQ + s * TILE + c * 16384, &maps.q, &bar_qf[s], c * 64, i * 128, hed, bat);
                     ++q_loads[s];
+                    q_issued[s] = q_loads[s];
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             for (int g = 0; ok && g < P.groups; ++g) {
+                if (a.stall && rp >= 2) {  // test hook: no copy after the CTA's first K/V tile pair
+                    ok = false;
+                    break;
+                }
                 const int blk = nxt;
                 nxt = blk_of(g + 1);
                 for (int kv = 0; kv < 2; ++kv) {  // K then V of the group
@@ -542,7 +558,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 if (t + 1 < n) load_meta(t + 1);
                 const bool masked = tail_k >= 0;
-                if (!mbar_wait(&bar_sf[s], s_uses & 1, wc, 0x208)) { ok = false; break; }
+                // warp-uniform outcome: the lanes go on to warp-collective tcgen05 loads
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar_sf[s], s_uses & 1, wc, 0x208))) { ok = false; break; }
                 ++s_uses;
                 tc_fence_after();
                 uint32_t v[2][32];
@@ -646,7 +663,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             // epilogue: the row sum is split over the two half-warps
             l += __shfl_xor_sync(0xffffffffu, l, 16);
-            if (!mbar_wait(&bar_of[s], o_uses & 1, wc, 0x209)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar_of[s], o_uses & 1, wc, 0x209))) { ok = false; break; }
             ++o_uses;
             tc_fence_after();
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
@@ -684,6 +701,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(&bar_kvf[q % ST], (q / ST) & 1) &&
                        globaltimer_ns() - t0 < a.wait_ns) {
+                }
+            }
+            for (int s = 0; s < 2; ++s) {  // the last Q load of each row slot
+                if (q_issued[s] == 0) continue;
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&bar_qf[s], (q_issued[s] - 1) & 1) && globaltimer_ns() - t0 < a.wait_ns) {
                 }
             }
         }

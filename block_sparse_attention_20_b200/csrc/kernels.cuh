@@ -62,6 +62,7 @@ struct ScoreArgs {
     float2 *mz;    // [heads*MC][nchunk] (max, sum) of each chunk in base 2
     WsHeader *hdr;
     uint64_t wait_ns;
+    int stall;     // test hook: the copy producer stops after its first tile
 };
 struct ScoreMaps {
     CUtensorMap a;  // fp16 scaled centroids [heads][MC][D], box (64, 128, 1)
@@ -162,6 +163,7 @@ struct AttnArgs {
     float *lse;        // optional [B*H][N]
     WsHeader *hdr;
     uint64_t wait_ns;
+    int stall;         // test hook: the copy producer stops after its first K/V tile pair
 };
 struct AttnMaps {
     CUtensorMap q;  // (D, N, H, B), box (64, 128, 1, 1)

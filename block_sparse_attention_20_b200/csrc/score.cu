@@ -119,9 +119,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     // this CTA's key tiles: [kt0, kt0 + ntl)
     const int kt0 = chunk * a.chunk_tiles;
     const int ntl = min(a.chunk_tiles, a.nT - kt0);
-    // a bounded wait elsewhere already gave up: do not start more work
-    if (a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT))
-        return;
+    __shared__ int skip_s;
+    // a bounded wait elsewhere already gave up: do not start more work.  One
+    // read, shared by the whole CTA, so every role takes the same decision
+    if (threadIdx.x == 0)
+        skip_s = a.hdr && (*reinterpret_cast<volatile uint32_t *>(&a.hdr->status) & ABATT_DEVFLAG_TIMEOUT);
+    __syncthreads();
+    if (skip_s) return;
     const WaitCtx wc{&abort_s, a.hdr, a.wait_ns};
 
     if (threadIdx.x == 0) {
@@ -158,6 +162,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             for (int c = 0; c < CH; ++c) tma_load_3d(sA + c * 16384, &maps.a, &bar_a, c * 64, mt * 128, hd);
             for (int i = 0; i < ntl; ++i) {
                 const int s = i % ST;
+                if (a.stall && i >= 1) break;  // test hook: no copy after the CTA's first key tile
                 if (i >= ST && !mbar_wait(&bar_kempty[s], ((i / ST) - 1) & 1, wc, 0x101)) break;
                 mbar_arrive_expect_tx(&bar_kfull[s], TILE);
                 for (int c = 0; c < CH; ++c)
@@ -225,7 +230,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         for (int i = e; i < ntl; i += kScoreEpi) {
             const int kt = kt0 + i, use = i / kScoreEpi;
-            if (!mbar_wait(&bar_sfull[e], use & 1, wc, 0x105)) break;
+            // warp-uniform outcome: the lanes go on to warp-collective tcgen05 loads
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar_sfull[e], use & 1, wc, 0x105))) break;
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + e * 128;
             const int nvalid = min(128, a.N - kt * 128);  // < 128 only on the sequence's last tile

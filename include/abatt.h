@@ -179,17 +179,38 @@ abatt_status abatt_sample(const float *p, const abatt_shape *shape, const abatt_
  * block b shifted by logw_b:
  *   O[q] = sum_t e^{l_t} v_t / sum_t e^{l_t},  l_t = s q.k_t + logw_{b(t)}.
  * Each row's list must be strictly ascending (as abatt_sample writes it).
- * Blocks are gathered from K/V into 128-key tensor-core tiles; two
- * neighbouring query blocks (rows 2p, 2p+1) share the gathers of the union
- * of their lists, each masking the blocks it did not draw.  An empty list
- * gives O = 0 (and lse = -inf).  lse (optional, NULL to skip): fp32
- * [B][H][N], natural-log sum of exponentials per query.  Indices outside
- * [0, nK) or out of order are skipped and flagged ABATT_DEVFLAG_BADLIST. */
+ * Blocks are gathered from K/V into 128-key tensor-core tiles.  Two
+ * neighbouring query blocks (rows 2p, 2p+1 of a head) run together: their
+ * lists are laid out as [blocks both drew | row 2p only | row 2p+1 only]; each
+ * row walks exactly its own blocks ([both | its own]) in tiles of 128/kv_block
+ * blocks, so no tile holds a block the row did not draw, and the tiles that
+ * lie wholly inside the shared segment are gathered once for both rows.  An
+ * empty list gives O = 0 (and lse = -inf).  lse (optional, NULL to skip):
+ * fp32 [B][H][N], natural-log sum of exponentials per query.  Indices outside
+ * [0, nK) or out of order are skipped and flagged ABATT_DEVFLAG_BADLIST.
+ * This is abatt_attention_plan followed by abatt_attention_planned. */
 abatt_status abatt_attention(const void *Q, const void *K, const void *V,
                              const abatt_shape *shape, const abatt_config *cfg,
                              const int32_t *counts, const int32_t *idx, const float *logw,
                              int capacity, void *O, float *lse, void *workspace,
                              size_t workspace_bytes, void *stream);
+
+/* The two launches of abatt_attention, for callers that time or repeat them
+ * separately.  abatt_attention_plan clears the workspace status word and
+ * lays every pair's lists out in the ATTENTION workspace (segment lengths,
+ * the pair's block array, each row's base-2 log-weights in its walking
+ * order); abatt_attention_planned runs the gather-attention kernel from that
+ * plan and does not clear the status word.  The plan stays valid while the
+ * workspace is not reused by another call; Q, K, V may change between
+ * planned calls.  Arguments as for abatt_attention. */
+abatt_status abatt_attention_plan(const abatt_shape *shape, const abatt_config *cfg,
+                                  const int32_t *counts, const int32_t *idx, const float *logw,
+                                  int capacity, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+abatt_status abatt_attention_planned(const void *Q, const void *K, const void *V,
+                                     const abatt_shape *shape, const abatt_config *cfg, void *O,
+                                     float *lse, void *workspace, size_t workspace_bytes,
+                                     void *stream);
 
 /* The whole path: select -> sample -> attention, on one stream, with p and the
  * lists kept in the workspace (capacity nK, so no row can overflow). */
@@ -219,21 +240,52 @@ abatt_status abatt_forward_intermediates(void *workspace, const abatt_shape *sha
  * rejected with ABATT_ERR_UNSUPPORTED before any launch (the scratch needed
  * is abatt_workspace_size(ABATT_CALL_ATTENTION, ...)).
  *
- * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  Every
- * call on a device shares the one array and leaves its contents behind:
- * calls that may overlap on the GPU (different streams without ordering, or
- * concurrent host threads) race on it and must be serialised by the caller.
- * The call allocates and frees nothing.
+ * The array's device address is looked up with cudaGetSymbolAddress the
+ * first time the call runs in a CUDA context (the current device's), and
+ * cached for that context only: a call from another context (after
+ * cudaDeviceReset, or one a host created with the driver API) looks it up
+ * again.  Make the first call in each context before any stream capture.
+ * Every call on a device shares the one array and leaves its contents
+ * behind: calls that may overlap on the GPU (different streams without
+ * ordering, or concurrent host threads) race on it and must be serialised by
+ * the caller.  The call allocates and frees nothing.
  *
- * dev_status (device pointer, NULL to skip) receives the ABATT_DEVFLAG_*
- * bits of this call, asynchronously on `stream`. */
+ * dev_status (device pointer, NULL to skip): once the arguments pass the
+ * host checks, it is set to ABATT_NOALLOC_STATUS_PENDING (all bits) on
+ * `stream`, and replaced by the ABATT_DEVFLAG_* bits of this call when every
+ * launch of the call was enqueued; if the call returns an error after that
+ * point, it keeps the PENDING value. */
+#define ABATT_NOALLOC_STATUS_PENDING 0xFFFFFFFFu
 #define ABATT_NOALLOC_SCRATCH_BYTES (64u << 20)
 abatt_status abatt_attention_noalloc(const void *Q, const void *K, const void *V,
                                      const abatt_shape *shape, const abatt_config *cfg,
                                      const int32_t *counts, const int32_t *idx, const float *logw,
                                      int capacity, void *O, float *lse, uint32_t *dev_status,
                                      void *stream);
+
+/* Test hooks (no counterpart in the paper).  They let the tests drive the
+ * failure path of the bounded device waits without faulting a GPU, and check
+ * the FMA-pipe exponential the kernels use, against CUDA's exp2f.
+ *   abatt_test_set(ABATT_TEST_WAIT_NS, ns): limit of every bounded wait of
+ *        later calls, in nanoseconds (0 restores the default, 0.5 s).
+ *   abatt_test_set(ABATT_TEST_STALL, mask): the copy producer of the
+ *        attention kernel (bit ABATT_TEST_STALL_ATTENTION) or of the scoring
+ *        kernel (ABATT_TEST_STALL_SCORE) stops after its first tile, so the
+ *        waits for later tiles run out: the call sets ABATT_DEVFLAG_TIMEOUT,
+ *        its CTAs drain what they issued, free tensor memory and return.  0
+ *        turns it off.
+ * Process-wide; not safe against calls running concurrently on other host
+ * threads.  ABATT_ERR_INVALID_ARG for an unknown hook. */
+enum { ABATT_TEST_WAIT_NS = 1, ABATT_TEST_STALL = 2 };
+#define ABATT_TEST_STALL_ATTENTION 0x1u
+#define ABATT_TEST_STALL_SCORE 0x2u
+abatt_status abatt_test_set(int hook, uint64_t value);
+
+/* y[i] = 2^x[i] through the kernels' FMA-pipe polynomial of the given degree
+ * (3 or 4): Cody-Waite reduction x = j + f and a minimax polynomial for 2^f
+ * with constant term 1; inputs at or below -127 give +0.  x and y are device
+ * fp32 arrays of n elements; asynchronous on `stream`. */
+abatt_status abatt_test_exp2_poly(const float *x, float *y, int64_t n, int degree, void *stream);
 
 /* Synchronously copy the device status word at the start of `workspace` to
  * *flags (ABATT_DEVFLAG_* bits) after `stream` drains.  Returns

@@ -58,11 +58,11 @@ def _load():
         lib.orc_inclusion.argtypes = [P, i32, i64, P, P, P, P, P]
         lib.orc_topk.argtypes = [P, i64, i32, i32, i32, i32, P, P, P]
         lib.orc_sample.argtypes = [P, i32, i32, i32, i32, i32, P, i64, i32, u64, i32, i32,
-                                   P, P, P, P, i32]
+                                   P, P, P, P, i32, i32, i32]
         lib.orc_ht_attention.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, i64,
                                          P, P, P, i32, i32, i32, P, P, P, P]
         lib.orc_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, i32, f64,
-                                    u64, P, i64, i32, P, P, P, P, P]
+                                    u64, P, i64, i32, P, P, P, P, P, i32, i32]
         _lib = lib
         return lib
 
@@ -182,11 +182,13 @@ def inclusion(p_row, M):
 
 
 def sample(p, shape, rows, budget_bp, seed, Bq=128, Bk=16, capacity=None, nthreads=None,
-           paired=False):
+           paired=False, batch_offset=0, head_offset=0):
     """O4: SIP draw for the listed rows (p is fp32 [nrows, nK]).
 
     paired=True: common random numbers -- query blocks 2j and 2j+1 of a head
     draw with the same Philox counter (floor(i/2) in place of i).
+    batch_offset, head_offset: global index of the shape's first batch element
+    and head when it is a slice of a larger problem (the counter's words 3, 2).
 
     Returns counts [nrows], idx [nrows, cap], logw fp32 [nrows, cap],
     amb uint8 [nrows, cap] (1 where the fp32 rounding of -ln(pi) is too close
@@ -202,7 +204,8 @@ def sample(p, shape, rows, budget_bp, seed, Bq=128, Bk=16, capacity=None, nthrea
     amb = np.zeros((len(r), cap), dtype=np.uint8)
     rc = _check(_load().orc_sample(_ptr(p), B, H, N, Bq, Bk, _ptr(r), len(r), int(budget_bp),
                                    int(seed) & (2**64 - 1), cap, nthreads or default_threads(),
-                                   _ptr(counts), _ptr(idx), _ptr(logw), _ptr(amb), int(bool(paired))),
+                                   _ptr(counts), _ptr(idx), _ptr(logw), _ptr(amb), int(bool(paired)),
+                                   int(batch_offset), int(head_offset)),
                 "sample")
     return counts, idx, logw, amb, bool(rc == 1)
 
@@ -254,8 +257,11 @@ def ht_attention(Q, K, V, shape, rows, counts, idx, logw, Bq=128, Bk=16, scale=N
 
 
 def forward(Q, K, V, shape, rows, C, iters, budget_bp, seed, Bq=128, Bk=16, scale=None,
-            nthreads=None):
-    """Whole path for the listed rows.  Returns dict(p32, counts, idx, logw, O)."""
+            nthreads=None, batch_offset=0, head_offset=0):
+    """Whole path for the listed rows.  Returns dict(p32, counts, idx, logw, O).
+
+    batch_offset, head_offset: global index of the tensors' first batch
+    element and head when they are a slice of a larger problem."""
     B, H, N, d = shape
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     nK = -(-N // Bk)
@@ -268,5 +274,6 @@ def forward(Q, K, V, shape, rows, C, iters, budget_bp, seed, Bq=128, Bk=16, scal
     _check(_load().orc_forward(_ptr(_bits(Q)), _ptr(_bits(K)), _ptr(_bits(V)), B, H, N, d, Bq,
                                Bk, C, iters, int(budget_bp), scale, int(seed) & (2**64 - 1),
                                _ptr(r), len(r), nthreads or default_threads(), _ptr(p32),
-                               _ptr(counts), _ptr(idx), _ptr(logw), _ptr(O)), "forward")
+                               _ptr(counts), _ptr(idx), _ptr(logw), _ptr(O), int(batch_offset),
+                               int(head_offset)), "forward")
     return dict(p32=p32, counts=counts, idx=idx, logw=logw, O=O)

@@ -610,6 +610,8 @@ static int sample_row(const float *p, const geom_t *g, int beta, int h, int i,
                       int32_t *count, int32_t *idx, float *logw, uint8_t *amb,
                       int *overflow)
 {
+    /* beta and h enter the counter as global indices: the caller adds the
+       offsets of a slice of a larger problem */
     const int nK = g->nK;
     int64_t M = orc_budget_blocks(budget_bp, nK);
     int64_t *P = (int64_t *)malloc(sizeof(int64_t) * (size_t)nK);
@@ -658,7 +660,7 @@ typedef struct {
     const float *p;
     geom_t g;
     const int64_t *rows;
-    int budget_bp, capacity, paired;
+    int budget_bp, capacity, paired, b_off, h_off;
     uint64_t seed;
     int32_t *counts, *idx;
     float *logw;
@@ -672,24 +674,29 @@ static void smp_row(void *vctx, int64_t k)
     int beta, h, i, of = 0;
     if (decode_row(&c->g, c->rows[k], &beta, &h, &i)) { c->bad = 1; return; }
     size_t o = (size_t)k * c->capacity;
-    if (sample_row(c->p + (size_t)k * c->g.nK, &c->g, beta, h, i, c->budget_bp, c->seed,
+    if (sample_row(c->p + (size_t)k * c->g.nK, &c->g, beta + c->b_off, h + c->h_off, i, c->budget_bp, c->seed,
                    c->paired, c->capacity, c->counts + k, c->idx + o, c->logw + o,
                    c->amb ? c->amb + o : NULL, &of))
         c->bad = 1;
     if (of) __atomic_store_n(&c->overflow, 1, __ATOMIC_RELAXED);
 }
 
-/* p is [nrows][nK] (row k belongs to linear row id rows[k]).  Returns 1 if
- * some row had more draws than `capacity` (its list is truncated). */
+/* p is [nrows][nK] (row k belongs to linear row id rows[k]).  b_off, h_off:
+ * global index of the tensor's first batch element and head, when it is a
+ * slice of a larger problem (0 otherwise).  Returns 1 if some row had more
+ * draws than `capacity` (its list is truncated). */
 int orc_sample(const float *p, int B, int H, int N, int Bq, int Bk,
                const int64_t *rows, int64_t nrows, int budget_bp, uint64_t seed,
                int capacity, int nthreads,
-               int32_t *counts, int32_t *idx, float *logw, uint8_t *amb, int paired)
+               int32_t *counts, int32_t *idx, float *logw, uint8_t *amb, int paired,
+               int b_off, int h_off)
 {
     smp_ctx c;
     memset(&c, 0, sizeof c);
     if (make_geom(&c.g, B, H, N, 1, Bq, Bk)) return -1;
     if (!p || !rows || !counts || !idx || !logw || capacity < 0 || budget_bp < 0) return -1;
+    if (b_off < 0 || h_off < 0) return -1;
+    c.b_off = b_off; c.h_off = h_off;
     if (c.g.nK > 32767) return -1;
     c.p = p; c.rows = rows; c.budget_bp = budget_bp; c.capacity = capacity; c.seed = seed;
     c.counts = counts; c.idx = idx; c.logw = logw; c.amb = amb; c.paired = paired ? 1 : 0;
@@ -899,7 +906,7 @@ int orc_ht_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
 typedef struct {
     const uint16_t *Q, *K, *V;
     geom_t g;
-    int C, iters, budget_bp;
+    int C, iters, budget_bp, b_off, h_off;
     double scale;
     uint64_t seed;
     const int64_t *rows;
@@ -927,7 +934,7 @@ static void fwd_row(void *vctx, int64_t k)
         c->bad = 1;
     } else {
         for (int b = 0; b < nK; ++b) p32[b] = (float)p[b];
-        if (sample_row(p32, g, beta, h, i, c->budget_bp, c->seed, 0, nK, c->counts + k, idx,
+        if (sample_row(p32, g, beta + c->b_off, h + c->h_off, i, c->budget_bp, c->seed, 0, nK, c->counts + k, idx,
                        logw, NULL, &of))
             c->bad = 1;
         for (int s = 0; s < c->counts[k]; ++s) lwd[s] = (double)logw[s];
@@ -943,17 +950,21 @@ static void fwd_row(void *vctx, int64_t k)
 }
 
 /* Outputs per listed row: p32 [nrows][nK], counts [nrows], idx/logw
- * [nrows][nK] (capacity nK), O [nrows][Bq][d]. */
+ * [nrows][nK] (capacity nK), O [nrows][Bq][d].  b_off, h_off: global index
+ * of the tensors' first batch element and head (the sampler's counter). */
 int orc_forward(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                 int B, int H, int N, int d, int Bq, int Bk, int C, int iters,
                 int budget_bp, double scale, uint64_t seed,
                 const int64_t *rows, int64_t nrows, int nthreads,
-                float *p32, int32_t *counts, int32_t *idx, float *logw, double *O)
+                float *p32, int32_t *counts, int32_t *idx, float *logw, double *O,
+                int b_off, int h_off)
 {
     fwd_ctx c;
     memset(&c, 0, sizeof c);
     if (make_geom(&c.g, B, H, N, d, Bq, Bk)) return -1;
     if (C <= 0 || C > Bq || iters < 0 || budget_bp < 0 || c.g.nK > 32767) return -1;
+    if (b_off < 0 || h_off < 0) return -1;
+    c.b_off = b_off; c.h_off = h_off;
     if (!Q || !K || !V || !rows || !p32 || !counts || !idx || !logw || !O) return -1;
     c.Q = Q; c.K = K; c.V = V; c.C = C; c.iters = iters; c.budget_bp = budget_bp;
     c.scale = scale; c.seed = seed; c.rows = rows;

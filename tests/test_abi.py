@@ -151,3 +151,68 @@ def test_shape_of_follows_the_layout():
     assert (sh.B, sh.H, sh.N, sh.d) == (2, 5, 300, 64)
     sh = abatt._shape_of(q, abatt.Config())
     assert (sh.B, sh.H, sh.N, sh.d) == (2, 300, 5, 64)
+
+
+def test_host_side_rejections_of_the_attention_launches_and_test_hooks(L):
+    sh = abatt._Shape(1, 2, 256, 64)
+    cfg = abatt.Config()._c(64)
+    P = ctypes.c_void_p
+    ok = P(0x100000)
+    # plan: null lists, capacity < 1, missing workspace
+    assert L.abatt_attention_plan(ctypes.byref(sh), ctypes.byref(cfg), None, ok, ok, 16, ok, 1 << 30,
+                                  None) == 1
+    assert L.abatt_attention_plan(ctypes.byref(sh), ctypes.byref(cfg), ok, ok, ok, 0, ok, 1 << 30,
+                                  None) == 1
+    assert L.abatt_attention_plan(ctypes.byref(sh), ctypes.byref(cfg), ok, ok, ok, 16, None, 0,
+                                  None) == 4
+    # planned: null and misaligned tensors, small workspace
+    assert L.abatt_attention_planned(None, ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, None, ok,
+                                     1 << 30, None) == 1
+    assert L.abatt_attention_planned(P(0x1001), ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, None,
+                                     ok, 1 << 30, None) == 3
+    assert L.abatt_attention_planned(ok, ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, None, ok, 255,
+                                     None) == 4
+    # test hooks: unknown hook, bad degree, negative size
+    assert L.abatt_test_set(99, 0) == 1
+    assert L.abatt_test_exp2_poly(ok, ok, 16, 5, None) == 1
+    assert L.abatt_test_exp2_poly(None, ok, 16, 3, None) == 1
+    assert L.abatt_test_exp2_poly(ok, ok, -1, 3, None) == 1
+    # the no-alloc call: null inputs, then a shape beyond its scratch (before any device call)
+    assert L.abatt_attention_noalloc(None, ok, ok, ctypes.byref(sh), ctypes.byref(cfg), ok, ok, ok, 16,
+                                     ok, None, None, None) == 1
+    big = abatt._Shape(1, 40, 75600, 128)
+    assert L.abatt_attention_noalloc(ok, ok, ok, ctypes.byref(big), ctypes.byref(abatt.Config()._c(128)),
+                                     ok, ok, ok, 16, ok, None, None, None) == 2
+
+
+def test_binding_checks_buffer_shapes_dtypes_and_devices():
+    import torch
+
+    cpu = torch.device("cpu")
+    rows, cap = 6, 10
+    counts = torch.zeros(rows, dtype=torch.int32)
+    idx = torch.zeros((rows, cap), dtype=torch.int32)
+    logw = torch.zeros((rows, cap), dtype=torch.float32)
+    assert abatt._check_lists(counts, idx, logw, rows, cpu) == cap
+    with pytest.raises(ValueError, match="counts"):
+        abatt._check_lists(counts[:5], idx, logw, rows, cpu)
+    with pytest.raises(ValueError, match="idx"):
+        abatt._check_lists(counts, idx.long(), logw, rows, cpu)
+    with pytest.raises(ValueError, match="logw"):
+        abatt._check_lists(counts, idx, logw[:, :9], rows, cpu)
+    with pytest.raises(ValueError, match="capacity"):
+        abatt._check_lists(counts, idx[:, :0], logw[:, :0], rows, cpu)
+    with pytest.raises(ValueError, match="not contiguous"):
+        abatt._check_lists(counts, idx, torch.zeros((cap, rows)).t(), rows, cpu)
+    q = torch.zeros((1, 2, 300, 64), dtype=torch.bfloat16)
+    sh = abatt._shape_of(q, abatt.Config())
+    abatt._check_outputs(q, torch.zeros_like(q), torch.zeros((1, 2, 300)), sh)
+    with pytest.raises(ValueError, match="out"):
+        abatt._check_outputs(q, torch.zeros((1, 2, 299, 64), dtype=torch.bfloat16), None, sh)
+    with pytest.raises(ValueError, match="out"):
+        abatt._check_outputs(q, torch.zeros_like(q, dtype=torch.float32), None, sh)
+    with pytest.raises(ValueError, match="lse"):
+        abatt._check_outputs(q, None, torch.zeros((1, 2, 300), dtype=torch.float64), sh)
+    # Q, K, V must be CUDA bf16 tensors of one shape
+    with pytest.raises(ValueError):
+        abatt._check_qkv(q, q, q)  # CPU tensors

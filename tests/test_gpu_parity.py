@@ -77,7 +77,7 @@ def _rows_of(shape, Bq=128):
                                            (9001, 16, 800, 0.1)])
 def test_sample_bit_exact(nK, Bk, bp, conc):
     N = nK * Bk - (Bk // 2 if nK > 1 else 0)
-    shape = (1, 2, N, 64)
+    shape = (2 if nK in (4725, 256, 63) else 1, 2, N, 64)  # B = 2: the counter's batch word
     rows = _rows_of(shape)
     p = synth.random_probs(len(rows), nK, 1000 + nK, conc)
     # special rows: all zero, one-hot, NaN / negative / > 1 entries, uniform
@@ -125,13 +125,31 @@ def test_sample_topk_bit_exact(nK, bp, coarse):
 def test_sample_paired_bit_exact(nK, Bk, bp):
     # common random numbers: the counter's query-block word is i/2
     N = nK * Bk - Bk // 2
-    shape = (1, 2, N, 64)
+    shape = (2 if nK in (4725, 63) else 1, 2, N, 64)
     rows = _rows_of(shape)
     p = synth.random_probs(len(rows), nK, 3000 + nK, 0.2)
     cfg = abatt.Config(kv_block=Bk, budget_bp=bp, seed=0x1234ABCD5678EF90, draws=abatt.DRAWS_PAIRED)
     c, i, lw, ws = abatt.sample(torch.from_numpy(p).cuda(), shape, cfg)
     assert abatt.read_status(ws) == 0
     oc, oi, ol, oamb, _ = oracle.sample(p, shape, rows, bp, cfg.seed, Bk=Bk, paired=True)
+    _check_lists_exact(c.cpu().numpy(), i.cpu().numpy(), lw.cpu().numpy(), oc, oi, ol, oamb)
+
+
+@pytest.mark.parametrize("nK,b_off,h_off,paired", [(4725, 3, 5, False), (700, 1, 0, True), (9001, 0, 17, False)])
+def test_sample_slice_offsets_bit_exact(nK, b_off, h_off, paired):
+    # a call over a slice of a larger problem draws with global (batch, head)
+    # indices: the device against the oracle given the same offsets
+    Bk = 16
+    N = nK * Bk - Bk // 2
+    shape = (2, 2, N, 64)
+    rows = _rows_of(shape)
+    p = synth.random_probs(len(rows), nK, 5000 + nK, 0.15)
+    cfg = abatt.Config(kv_block=Bk, budget_bp=900, seed=0x0F1E2D3C4B5A6978, batch_offset=b_off, head_offset=h_off,
+                       draws=abatt.DRAWS_PAIRED if paired else abatt.DRAWS_INDEPENDENT)
+    c, i, lw, ws = abatt.sample(torch.from_numpy(p).cuda(), shape, cfg)
+    assert abatt.read_status(ws) == 0
+    oc, oi, ol, oamb, _ = oracle.sample(p, shape, rows, 900, cfg.seed, Bk=Bk, paired=paired,
+                                        batch_offset=b_off, head_offset=h_off)
     _check_lists_exact(c.cpu().numpy(), i.cpu().numpy(), lw.cpu().numpy(), oc, oi, ol, oamb)
 
 
@@ -276,6 +294,26 @@ def test_attention_large_logweights_and_scale():
     _attn_check(Q, K, V, shape, 16, rows, c, i, lw, scale=0.2)
 
 
+def test_attention_plan_then_planned_is_attention():
+    # the two launches separately give the bits of the one call; the plan can
+    # be run again on other values of Q, K, V
+    shape = (2, 3, 1000, 128)
+    Q, K, V = (synth.random_bf16(shape, s).cuda() for s in (61, 62, 63))
+    rows, c, i, lw = _random_lists(shape, 16, 1500, 64)
+    counts, idx, logw = (torch.from_numpy(x).cuda() for x in (c, i, lw))
+    cfg = abatt.Config(kv_block=16)
+    ref, ref_lse = abatt.attention(Q, K, V, counts, idx, logw, cfg, want_lse=True)
+    ws = torch.empty(abatt.workspace_size(abatt.CALL_ATTENTION, shape, cfg), dtype=torch.uint8, device="cuda")
+    abatt.attention_plan(shape, counts, idx, logw, cfg, workspace=ws)
+    for _ in range(2):
+        O, lse = abatt.attention_planned(Q, K, V, cfg, workspace=ws, want_lse=True)
+        torch.cuda.synchronize()
+        assert abatt.read_status(ws) == 0
+        assert torch.equal(O, ref) and torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32))
+    O2 = abatt.attention_planned(Q, K, K, cfg, workspace=ws)  # V replaced by K
+    assert torch.equal(O2, abatt.attention(Q, K, K, counts, idx, logw, cfg))
+
+
 def test_attention_empty_rows_and_bad_index():
     shape = (1, 2, 512, 64)
     Q, K, V = (synth.random_bf16(shape, s) for s in (10, 11, 12))
@@ -308,7 +346,22 @@ def test_attention_empty_rows_and_bad_index():
 
 # --------------------------------------------------------------------------- selector
 
-def _select_check(Q, K, shape, C, I, Bk, rows_check=None, coarse=False):
+# Element-wise tolerance of the block probabilities.  The scoring GEMM takes
+# the scaled centroids rounded to fp16 (relative error <= 2^-11 per
+# coordinate; the keys are exact in fp16), so a base-2 logit x = c'.k moves by
+# at most 2^-11 * sum_i |c'_i k_i|, below 0.02 on these inputs, and a block's
+# softmax mass by at most ~ln 2 * 2 * 0.02 relative (its own logits and the
+# normaliser): P_RTOL.  P_ATOL covers blocks whose mass is at the fp32 floor.
+P_RTOL = 3e-2
+P_ATOL = 1e-7
+
+
+def _select_check(Q, K, shape, C, I, Bk, rows_check=None, coarse=False, report=None):
+    """Selector against the oracle.  k-means may flip a near-tie in fp32 (the
+    GPU drops |q|^2 and rounds the products differently): rows whose cluster
+    sizes differ from the oracle's are counted and reported (at most 5 %
+    allowed); every other row is held to the centroid, the element-wise p and
+    the per-row L1 tolerances.  Returns p and the flip share."""
     cfg = abatt.Config(kv_block=Bk, clusters=C, kmeans_iters=I,
                        scoring=abatt.SCORE_BLOCK_MEANS if coarse else abatt.SCORE_KEYS)
     p, cent, sizes = abatt.select(Q.cuda(), K.cuda(), cfg, want_centroids=True)
@@ -316,14 +369,23 @@ def _select_check(Q, K, shape, C, I, Bk, rows_check=None, coarse=False):
     rows = _rows_of(shape) if rows_check is None else np.asarray(rows_check)
     ocent, osz, _ = oracle.kmeans(Q, shape, rows, C, I)
     same_sizes = np.all(sizes[rows] == osz, axis=1)
-    assert same_sizes.mean() >= 0.95
+    flips = 1.0 - float(same_sizes.mean())
+    assert flips <= 0.05, flips
     ok = same_sizes
     assert np.max(np.abs(cent[rows][ok] - ocent[ok])) <= 1e-4 * max(1.0, np.abs(ocent).max())
     p64, p32 = oracle.block_probs(Q, K, shape, rows, C, I, Bk=Bk, coarse=coarse)
     assert np.allclose(p.sum(1), 1.0, atol=2e-4)
-    l1 = np.abs(p[rows][ok] - p64[ok]).sum(1)
+    got, ref = p[rows][ok], p64[ok]
+    l1 = np.abs(got - ref).sum(1)
     assert np.max(l1) <= 2e-3, np.max(l1)
-    return p
+    err = np.abs(got - ref)
+    bad = err > P_ATOL + P_RTOL * ref
+    assert not bad.any(), (int(bad.sum()), float((err / np.maximum(ref, 1e-30))[bad].max()))
+    if report is not None:
+        big = ref > 1e-4
+        report.update(flips=flips, rows=len(rows), max_l1=float(np.max(l1)),
+                      max_rel=float((err[big] / ref[big]).max()) if big.any() else 0.0)
+    return p, flips
 
 
 def test_select_tiny():
@@ -372,6 +434,19 @@ def test_select_block_means_ragged(N, Bk, C):
     w = synth.WAN_1_3B.with_(H=2, N=N, grid=(1, 20, N // 20))
     Q, K, V = synth.generate(w)
     _select_check(Q, K, w.shape, C, 5, Bk, coarse=True)
+
+
+def test_select_block_means_key_range_split_over_ctas(capsys):
+    # nK = 6,144 key blocks = 48 column tiles, one head: 48 centroid tiles of
+    # 128 rows fill a 148-SM GPU only when the block range is split into
+    # chunks (two here), which the second pass merges
+    w = synth.WAN_1_3B.with_(H=1, N=98304, grid=(32, 48, 64))
+    Q, K, V = synth.generate(w)
+    rep = {}
+    rows = _rows_of(w.shape)[::3]
+    _select_check(Q, K, w.shape, 8, 5, 16, rows_check=rows, coarse=True, report=rep)
+    with capsys.disabled():
+        print(f"\nblock means, nK = 6144: {rep}")
 
 
 def test_select_block_means_d64_growing_keys():
@@ -560,21 +635,32 @@ def test_forward_wan1_3b_full():
     _forward_check(w, _rows_of(w.shape))
 
 
-def test_forward_hunyuan_sampled_rows():
-    # 118,800 tokens: 929 query blocks per head (odd, last block 16 rows)
+def _subsample(w, heads=None):
+    """All heads, every query block i = 0 (mod 16), plus the last one."""
+    H = w.H if heads is None else heads
+    qs = sorted(set(range(0, w.nQ, 16)) | {w.nQ - 1})
+    return np.array([h * w.nQ + i for h in range(H) for i in qs])
+
+
+def test_forward_hunyuan_subsample(capsys):
+    # 118,800 tokens, 24 heads: 929 query blocks per head (odd; the last holds
+    # 16 rows and is i = 928 = 58 * 16); 59 rows per head, 1,416 in all
     w = synth.HUNYUAN
-    heads = 4
-    nQ = w.nQ
-    rows = [h * nQ + i for h, i in [(0, 0), (0, nQ - 1), (1, 464), (2, 928), (3, 3)]]
-    _forward_check(w, rows, heads=heads)
+    rows = _subsample(w)
+    agree = _forward_check(w, rows)
+    with capsys.disabled():
+        print(f"\nhunyuanvideo: {len(rows)} rows, sampled-block agreement {agree:.5f}")
 
 
-def test_forward_wan14b_full_size_sampled_rows():
+def test_forward_wan14b_subsample(capsys):
+    # the benchmark's workload: 40 heads x (37 rows i = 0 mod 16 + the last,
+    # 80-row block) = 1,520 rows
     w = synth.WAN_14B
-    nQ = w.nQ
-    rows = [h * nQ + i for h, i in [(0, 0), (0, nQ - 1), (7, 100), (13, 295), (21, 1), (27, 400),
-                                    (33, 590), (39, 0), (39, 333), (39, nQ - 1)]]
-    _forward_check(w, rows)
+    rows = _subsample(w)
+    assert len(rows) == 1520
+    agree = _forward_check(w, rows)
+    with capsys.disabled():
+        print(f"\nwan14b-720p: {len(rows)} rows, sampled-block agreement {agree:.5f}")
 
 
 def test_host_pipeline_matches_one_forward():

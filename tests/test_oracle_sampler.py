@@ -215,3 +215,26 @@ def test_paired_draws_take_a_block_in_both_rows_with_the_smaller_probability():
     # and not the independent rate where the two differ noticeably
     gap = want - pis[0] * pis[1]
     assert np.all(both[gap > 0.1] / nseed > (pis[0] * pis[1])[gap > 0.1] + 0.05)
+
+
+def test_slice_with_offsets_draws_what_the_whole_problem_draws():
+    # the counter carries global (batch, head) indices: heads [1, 3) of batch 1
+    # of a 2 x 3-head problem, drawn as a 1 x 2-head tensor with
+    # batch_offset=1, head_offset=1, give the whole problem's lists
+    B, H, N, Bk = 2, 3, 4000, 16
+    nK, nQ = -(-N // Bk), -(-N // 128)
+    rows = np.arange(B * H * nQ)
+    p = synth.random_probs(len(rows), nK, 808, 0.2)
+    whole = oracle.sample(p, (B, H, N, 64), rows, 900, 4242, Bk=Bk)
+    sel = np.array([(1 * H + h) * nQ + i for h in (1, 2) for i in range(nQ)])
+    part = oracle.sample(p[sel], (1, 2, N, 64), np.arange(2 * nQ), 900, 4242, Bk=Bk,
+                         batch_offset=1, head_offset=1)
+    assert np.array_equal(part[0], whole[0][sel])
+    for k, r in enumerate(sel):
+        L = whole[0][r]
+        assert np.array_equal(part[1][k, :L], whole[1][r, :L])
+        assert np.array_equal(part[2][k, :L], whole[2][r, :L])
+    # without the offsets the slice draws other blocks
+    plain = oracle.sample(p[sel], (1, 2, N, 64), np.arange(2 * nQ), 900, 4242, Bk=Bk)
+    assert any(not np.array_equal(plain[1][k, :plain[0][k]], whole[1][r, :whole[0][r]])
+               for k, r in enumerate(sel))
