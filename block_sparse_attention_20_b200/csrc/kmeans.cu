@@ -16,7 +16,7 @@
 //     rows are one more tensor-core product, onehot(assignment)^T . Q
 //     (16 x 128 times 128 x D, exact products, fp32 accumulation in the
 //     hardware's fixed order, so the result is deterministic); centroid =
-//     sum / size.
+//     sum * (1/size), written with its bf16 operand parts.
 //
 // Rules (open in the abstract, fixed here): C_eff = min(C, n) clusters;
 // centroid j starts at row floor(j*n/C_eff); squared Euclidean distance,
@@ -103,23 +103,24 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
             }
         }
         __syncthreads();
+        // a centroid coordinate and its tensor-core operands: bf16 high part and
+        // bf16 residual
+        auto put = [&](int j, int x, float c) {
+            cent[j * D + x] = c;
+            const __nv_bfloat16 h = __float2bfloat16_rn(c);
+            chi[j * LDQ + x] = h;
+            clo[j * LDQ + x] = __float2bfloat16_rn(c - __bfloat162float(h));
+        };
         for (int e = tid; e < CP * D; e += kKmThreads) {
             const int j = e / D, x = e % D;
-            cent[e] = j < ce ? __bfloat162float(qs[(j * n) / ce * LDQ + x]) : 0.0f;
+            put(j, x, j < ce ? __bfloat162float(qs[(j * n) / ce * LDQ + x]) : 0.0f);
         }
         __syncthreads();
 
         const int rounds = a.iters > 0 ? a.iters : 1;
         for (int it = 0; it < rounds; ++it) {
-            // ---- centroid operands: bf16 hi + lo, squared norms ----
-            for (int e = tid; e < CP * D; e += kKmThreads) {
-                const int j = e / D, x = e % D;
-                const float c = cent[e];
-                const __nv_bfloat16 h = __float2bfloat16_rn(c);
-                chi[j * LDQ + x] = h;
-                clo[j * LDQ + x] = __float2bfloat16_rn(c - __bfloat162float(h));
-            }
-            // squared norms: warp w takes centroids w, w+4, ...; lanes split the dimensions
+            // ---- squared norms of the centroids (operands were written with them) ----
+            // warp w takes centroids w, w+4, ...; lanes split the dimensions
             for (int j = warp; j < CP; j += 4) {
                 float s = 0.0f;
 #pragma unroll
@@ -251,11 +252,12 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                     if (j >= ce) continue;
                     const int c = cnt_s[j];
                     if (c == 0) continue;  // an empty cluster keeps its centroid
+                    const float inv = __frcp_rn((float)c);  // sum / size as sum * (1/size)
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
                         const int x = n0w + 8 * t + 2 * cq;
-                        cent[j * D + x] = acc[t][2 * h] / (float)c;
-                        cent[j * D + x + 1] = acc[t][2 * h + 1] / (float)c;
+                        put(j, x, __fmul_rn(acc[t][2 * h], inv));
+                        put(j, x + 1, __fmul_rn(acc[t][2 * h + 1], inv));
                     }
                 }
             }

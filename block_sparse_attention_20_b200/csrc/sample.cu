@@ -24,23 +24,24 @@ constexpr int kSampleThreads = 256;
 constexpr int kSampleWarps = kSampleThreads / 32;
 constexpr int kCacheMaxBlocks = 8192;  // weights cached in shared memory up to this nK
 
-// round-half-even(p * 2^48) for p clamped to [0, 1] (NaN and negatives -> 0),
-// from the float's exponent and mantissa with integer shifts only.
+// round-half-even(p * 2^48) for p clamped to [0, 1] (NaN and negatives -> 0).
+// The scaling by a power of two is exact in fp32 (subnormal inputs included:
+// the build keeps subnormals), and the conversion to int64 rounds half to
+// even, so this is the exact fixed-point value.
 __device__ __forceinline__ int64_t to_fixed48(float p) {
     if (!(p > 0.0f)) return 0;
     if (p >= 1.0f) return int64_t(1) << 48;
-    const uint32_t bits = __float_as_uint(p);
-    const int e = (int)(bits >> 23);                      // biased exponent, 0 for subnormals
-    const uint32_t m = (bits & 0x7fffffu) | (e ? 0x800000u : 0u);
-    // value = m * 2^(e' - 150) * 2^48 with e' = max(e, 1) (subnormals use 1)
-    const int sh = (e ? e : 1) - 150 + 48;                // left shift of m (negative: right)
-    if (sh >= 0) return (int64_t)m << sh;                 // exact, < 2^48 since p < 1
-    const int rs = -sh;
-    if (rs > 24) return 0;                                // m < 2^24 <= 2^(rs-1): below one half
-    const uint32_t q = m >> rs;
-    const uint32_t rem = m & ((1u << rs) - 1u);
-    const uint32_t half = 1u << (rs - 1);
-    return (int64_t)(q + ((rem > half || (rem == half && (q & 1u))) ? 1u : 0u));
+    return __float2ll_rn(__fmul_rn(p, 0x1p48f));
+}
+
+// ceil(T / R) for 0 < T < 2^53, R > 0: the double quotient is within 1/16 of
+// T / R (both operands are exact in double), so its ceiling is off by at most
+// one, which the exact integer test corrects.
+__device__ __forceinline__ int64_t ceil_div(int64_t T, int64_t R) {
+    int64_t q = (int64_t)ceil((double)T / (double)R);
+    if (q * R < T) ++q;
+    else if ((q - 1) * R >= T) --q;
+    return q;
 }
 
 // Philox4x32-10 (Salmon et al., SC 2011): ten rounds, published multipliers
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleAr
             for (int round = 0; round <= nK; ++round) {
                 R = a.M - in_s;
                 if (T == 0 || R <= 0) break;
-                const int64_t thr = (T + R - 1) / R;
+                const int64_t thr = ceil_div(T, R);
                 int64_t added = 0, added_w = 0;
                 for (int b = tid; b < nK; b += kSampleThreads) {
                     if (sat[b]) continue;
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleAr
 // stay in registers for every water-filling round, and one block-wide scan of
 // the per-thread counts places the drawn blocks in ascending order.
 template <int NT, int G>
-__global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
+__global__ void __launch_bounds__(NT, NT == 256 ? 3 : 1) sample_compact_reg_kernel(SampleArgs a) {
     constexpr int NW = NT / 32;
     constexpr int PER = 4 * G;  // blocks per thread (<= 32: the masks are 32-bit)
     // the row is staged through shared memory with coalesced loads; thread
@@ -383,19 +384,31 @@ __global__ void __launch_bounds__(NT) sample_compact_reg_kernel(SampleArgs a) {
 #pragma unroll
             for (int q = 0; q < NW; ++q) T += red_w[q];
             int64_t in_s = 0;
+            // the largest weight of this thread's run still outside S: a round
+            // with a higher threshold adds nothing here
+            int64_t wmax = 0;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) wmax = max(wmax, P[k]);
             for (int round = 0; round <= nK; ++round) {
                 R = a.M - in_s;
                 if (T == 0 || R <= 0) break;
-                const int64_t thr = (T + R - 1) / R;
+                const int64_t thr = ceil_div(T, R);
                 int cnt = 0;
                 int64_t w = 0;
+                if (wmax >= thr) {
+                    int64_t rest = 0;
 #pragma unroll
-                for (int k = 0; k < PER; ++k) {
-                    if (!((sat >> k) & 1u) && P[k] >= thr) {
-                        sat |= 1u << k;
-                        ++cnt;
-                        w += P[k];
+                    for (int k = 0; k < PER; ++k) {
+                        if ((sat >> k) & 1u) continue;
+                        if (P[k] >= thr) {
+                            sat |= 1u << k;
+                            ++cnt;
+                            w += P[k];
+                        } else {
+                            rest = max(rest, P[k]);
+                        }
                     }
+                    wmax = rest;
                 }
                 // count and weight reduced together: one barrier pair per round
 #pragma unroll
