@@ -264,7 +264,6 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
     sa.last_weight = coarse ? (float)(g.N - (g.nK - 1) * g.Bk) / (float)g.Bk : 1.0f;
     score_chunks(sa.nT, ((int)MC + 127) / 128 * g.heads, sms, &sa.nchunk, &sa.chunk_tiles);
     sa.r = at<float>(ws, L.r);
-    sa.r16 = at<__half>(ws, L.r);  // the per-key rule's fp16 view of the same region
     sa.mref = at<float>(ws, L.mref);
     sa.mz = at<float2>(ws, L.mz);
     sa.hdr = at<WsHeader>(ws, L.hdr);
@@ -287,7 +286,7 @@ abatt_status run_select(const void *Q, const void *K, const Geom &g, const abatt
 
     CombineArgs ca;
     ca.rows = g.rows; ca.C = g.C; ca.nK = g.nK; ca.nT = sa.nT; ca.ldr = sa.ldr; ca.Bk = g.Bk;
-    ca.r = sa.r; ca.r16 = sa.r16; ca.mref = sa.mref; ca.weight = ka.weight; ca.mz = sa.mz; ca.p = p;
+    ca.r = sa.r; ca.mref = sa.mref; ca.weight = ka.weight; ca.mz = sa.mz; ca.p = p;
     ca.nchunk = sa.nchunk;
     return cuda_status(coarse ? launch_combine_cols(ca, sms, st) : launch_combine(ca, sms, st));
 }

@@ -57,9 +57,7 @@ struct ScoreArgs {
     int C;
     const float *weight;  // [heads*MC] n_j / n (mode 2)
     float *p;             // [heads*MC/C][N] (mode 2)
-    float *r;      // [heads*MC][ldr]: coarse scoring (Bk == 1), mode 0
-    __half *r16;   // [heads*MC][ldr]: per-key scoring -- fp16 block sums, each below 2^15
-                   // (relative to the tile's reference maximum; larger ones take the exact path)
+    float *r;      // [heads*MC][ldr]
     float *mref;   // [heads*MC][nT], running maximum within the tile's chunk
     float2 *mz;    // [heads*MC][nchunk] (max, sum) of each chunk in base 2
     WsHeader *hdr;
@@ -91,7 +89,6 @@ struct CombineArgs {
     int64_t rows;  // query blocks
     int C, nK, nT, ldr, Bk, nchunk;
     const float *r, *mref, *weight;
-    const __half *r16;  // per-key block sums (fp16), read by launch_combine
     const float2 *mz;
     float *p;      // [rows][nK]
 };

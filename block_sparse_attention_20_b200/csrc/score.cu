@@ -15,9 +15,8 @@
 // the row's running maximum and sum them per key block, two values per
 // packed fp32 instruction, with a fixed share of the exponentials on the FMA
 // pipe (polynomial) and the rest on the special-function unit.  The partial
-// block sums of a tile are written (fp16: 11 significant bits, each sum below
-// 2^15) with the reference maximum they were taken against, so no second pass
-// over the keys is needed.
+// block sums of a tile are written with the reference maximum they were
+// taken against, so no second pass over the keys is needed.
 //
 // combine_kernel: one CTA per query block:
 //   p_b = sum_j (n_j/n) * r_{j,b} * 2^(mref_{j,T(b)} - m_j) / Z_j
@@ -82,21 +81,16 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// The BPT block sums of one tile as fp16 (BPT = 128/Bk: 8, 4, 2 or 1 values).
 template <int BPT>
-__device__ __forceinline__ void store_blocks(__half *dst, const float (&bs)[BPT]) {
-    if constexpr (BPT == 1) {
-        dst[0] = __float2half_rn(bs[0]);
-    } else {
-        uint32_t w[BPT / 2];
+__device__ __forceinline__ void store_blocks(float *dst, const float (&bs)[BPT]) {
+    if constexpr (BPT % 4 == 0) {
 #pragma unroll
-        for (int k = 0; k < BPT; k += 2) {
-            const __half2 h = __floats2half2_rn(bs[k], bs[k + 1]);
-            w[k / 2] = *reinterpret_cast<const uint32_t *>(&h);
-        }
-        if constexpr (BPT == 8) *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-        else if constexpr (BPT == 4) *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
-        else *reinterpret_cast<uint32_t *>(dst) = w[0];
+        for (int k = 0; k < BPT; k += 4)
+            *reinterpret_cast<float4 *>(dst + k) = make_float4(bs[k], bs[k + 1], bs[k + 2], bs[k + 3]);
+    } else if constexpr (BPT == 2) {
+        *reinterpret_cast<float2 *>(dst) = make_float2(bs[0], bs[1]);
+    } else {
+        dst[0] = bs[0];
     }
 }
 
@@ -440,9 +434,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     float big = 0.0f;
 #pragma unroll
                     for (int k = 0; k < BPT; ++k) big = fmaxf(big, bs[k]);
-                    // block sums are stored in fp16: past 2^15 the tile is redone
-                    // against its own maximum (sums <= 16 then)
-                    redo = __any_sync(0xffffffffu, !(big < 0x1p15f));
+                    redo = __any_sync(0xffffffffu, !(big < 0x1p80f));
                 }
                 if (redo) exact();
                 // leave -m_run in the buffer for its next tile, then free it
@@ -458,7 +450,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 #pragma unroll
                 for (int k = 0; k < BPT; ++k) Z += bs[k];
                 if (valid) {
-                    store_blocks<BPT>(a.r16 + gr * a.ldr + (int64_t)kt * BPT, bs);
+                    store_blocks<BPT>(a.r + gr * a.ldr + (int64_t)kt * BPT, bs);
                     a.mref[gr * a.nT + kt] = m_run;
                 }
             }
@@ -547,18 +539,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
                     if (j < a.C) {
                         const int64_t cj = row * a.C + j;
                         mr[u] = __ldg(a.mref + cj * a.nT + T);
-                        const __half *rr = a.r16 + cj * a.ldr + (int64_t)T * BPT;
-                        if constexpr (BPT == 8) {
-                            const uint4 q = __ldg(reinterpret_cast<const uint4 *>(rr));
-                            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+                        const float *rr = a.r + cj * a.ldr + (int64_t)T * BPT;
+                        if constexpr (BPT % 4 == 0) {
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[k]));
-                                rv[u][2 * k] = f.x; rv[u][2 * k + 1] = f.y;
+                            for (int k = 0; k < BPT; k += 4) {
+                                const float4 q = __ldg(reinterpret_cast<const float4 *>(rr + k));
+                                rv[u][k] = q.x; rv[u][k + 1] = q.y; rv[u][k + 2] = q.z; rv[u][k + 3] = q.w;
                             }
                         } else {
 #pragma unroll
-                            for (int k = 0; k < BPT; ++k) rv[u][k] = __half2float(rr[k]);
+                            for (int k = 0; k < BPT; ++k) rv[u][k] = __ldg(rr + k);
                         }
                     }
                 }
