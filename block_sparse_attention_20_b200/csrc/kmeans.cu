@@ -12,7 +12,8 @@
 //     about 16 significant bits of the centroid; warp w takes rows
 //     32w..32w+31; the argmin (ties to the lower index) is reduced across the
 //     four lanes that share a row;
-//   - update: cluster sizes from warp ballots; the per-cluster sums of the
+//   - update: cluster sizes from warp ballots (each warp counts its own 32
+//     rows right after assigning them); the per-cluster sums of the
 //     rows are one more tensor-core product, onehot(assignment)^T . Q
 //     (16 x 128 times 128 x D, exact products, fp32 accumulation in the
 //     hardware's fixed order, so the result is deterministic); centroid =
@@ -78,7 +79,6 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
     __shared__ float cnorm[kMaxC];
     __shared__ int assign_s[128];
     __shared__ int wcnt_s[4][kMaxC];
-    __shared__ int cnt_s[kMaxC];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, cq = lane & 3;  // mma fragment coordinates
@@ -197,18 +197,15 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                     assign_s[r0 + g + 8] = (r0 + g + 8) < n ? besti[m][1] : -1;
                 }
             }
-            __syncthreads();
-
-            // ---- cluster sizes: ballots of this warp's rows, summed over warps ----
+            // ---- cluster sizes of this warp's 32 rows (ballots), before the barrier ----
+            __syncwarp();
             {
-                const int best = assign_s[tid];
+                const int best = assign_s[tid];  // row tid belongs to this warp
                 for (int j = 0; j < ce; ++j) {
                     const uint32_t m = __ballot_sync(0xffffffffu, best == j);
                     if (lane == 0) wcnt_s[warp][j] = __popc(m);
                 }
             }
-            __syncthreads();
-            if (tid < ce) cnt_s[tid] = wcnt_s[0][tid] + wcnt_s[1][tid] + wcnt_s[2][tid] + wcnt_s[3][tid];
             __syncthreads();
             if (a.iters == 0) break;  // sizes from the seeds, no update
 
@@ -250,7 +247,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                 for (int h = 0; h < 2; ++h) {
                     const int j = g + 8 * h;
                     if (j >= ce) continue;
-                    const int c = cnt_s[j];
+                    const int c = wcnt_s[0][j] + wcnt_s[1][j] + wcnt_s[2][j] + wcnt_s[3][j];
                     if (c == 0) continue;  // an empty cluster keeps its centroid
                     const float inv = __frcp_rn((float)c);  // sum / size as sum * (1/size)
 #pragma unroll
@@ -274,7 +271,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
             if (a.cent_out) a.cent_out[o] = c;
         }
         if (tid < C) {
-            const int c = tid < ce ? cnt_s[tid] : 0;
+            const int c = tid < ce ? wcnt_s[0][tid] + wcnt_s[1][tid] + wcnt_s[2][tid] + wcnt_s[3][tid] : 0;
             a.weight[row * C + tid] = (float)c / (float)n;
             if (a.sizes_out) a.sizes_out[row * C + tid] = c;
         }
