@@ -763,3 +763,32 @@ def test_sip_and_topk_error_against_dense_attention(capsys):
               f"keep-all {err['keep-all']:.5f}")
     assert err["keep-all"] <= REL_L2
     assert all(np.isfinite(v) for v in err.values())
+
+
+def test_sweep_error_against_dense_oracle(capsys):
+    # the sweep's accuracy column against dense float64 attention (O1), on a
+    # row subsample of the N = 8,192 sweep workload (24 heads, drawn on the GPU):
+    # every budget and two block sizes, through the whole path.  Reported (pytest
+    # -s), not judged, except that keep-all must reproduce dense attention and
+    # the error must not grow with the budget by more than noise
+    N = 8192
+    w0 = synth.sweep(N, 100, 16)
+    Q, K, V = synth.generate_on_device(w0, torch.device("cuda"))
+    Qc, Kc, Vc = Q.cpu(), K.cpu(), V.cpu()
+    rows = np.array([h * w0.nQ + i for h in range(0, 24, 4) for i in (0, 21, 42, 63)])
+    dense = oracle.dense_attention(Qc, Kc, Vc, w0.shape, rows)
+    table = {}
+    for Bk in (16, 64):
+        for bpct in (5, 10, 25, 50, 100):
+            w = synth.sweep(N, bpct, Bk)
+            cfg = cfg_of(w)
+            O = abatt.forward(Q, K, V, cfg).float().cpu().numpy()
+            got = np.stack([O[0, r // w.nQ, (r % w.nQ) * 128:(r % w.nQ + 1) * 128] for r in rows])
+            table[(Bk, bpct)] = _rel_l2(got, dense)
+    with capsys.disabled():
+        print("\nsweep N=8192, rel L2 of O against dense float64 attention (24 query blocks):")
+        for Bk in (16, 64):
+            print(f"  Bk={Bk}: " + ", ".join(f"{b} %: {table[(Bk, b)]:.4f}" for b in (5, 10, 25, 50, 100)))
+    for Bk in (16, 64):
+        assert table[(Bk, 100)] <= REL_L2
+        assert table[(Bk, 50)] <= table[(Bk, 5)] + 0.05
