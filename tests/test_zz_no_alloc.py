@@ -54,6 +54,20 @@ def test_noalloc_matches_attention_twice(shape, Bk):
         assert int(status.item()) == 0
         assert torch.equal(outs[k], ref)
         assert torch.equal(lses[k].view(torch.int32), ref_lse.view(torch.int32))
+    # and it is the method's attention: rows of the output against the float64 oracle
+    B, H, N, d = shape
+    nQ = -(-N // 128)
+    rows = np.array([0, nQ - 1, B * H * nQ - 1])
+    c, i, lw = (t.cpu().numpy() for t in (counts, idx, logw))
+    o5, _ = oracle.ht_attention(Q.cpu(), K.cpu(), V.cpu(), shape, rows, c[rows], i[rows], lw[rows], Bk=Bk)
+    got = np.zeros_like(o5)
+    Of = outs[1].float().cpu().numpy()
+    for k, r in enumerate(rows):
+        bh, q = divmod(int(r), nQ)
+        n = min(128, N - q * 128)
+        got[k, :n] = Of[bh // H, bh % H, q * 128:q * 128 + n]
+    assert np.linalg.norm(got - o5) / np.linalg.norm(o5) <= 5e-3
+    assert np.max(np.abs(got - o5)) <= 2e-2
 
 
 def test_noalloc_status_reads_pending_until_the_call_completes():
