@@ -66,7 +66,7 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 }
 
 // ============================== pair union ======================================
-constexpr int kUnionThreads = 256;
+constexpr int kUnionThreads = 128;
 
 // Entry j of a list is used if it is a block index and exceeds the previous
 // entry (when that one is a block index itself).
@@ -767,7 +767,7 @@ cudaError_t launch_pair_union(const PairArgs &a, int num_sms, cudaStream_t strea
     if (a.pairs < 1) return cudaSuccess;
     const size_t smem = sizeof(uint32_t) * 5 * (size_t)((a.nK + 31) / 32);
     int64_t grid = a.pairs;
-    if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
+    if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
     pair_union_kernel<<<(unsigned)grid, kUnionThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
