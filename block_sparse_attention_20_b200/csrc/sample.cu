@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_compact_kernel(SampleAr
 // stay in registers for every water-filling round, and one block-wide scan of
 // the per-thread counts places the drawn blocks in ascending order.
 template <int NT, int G>
-__global__ void __launch_bounds__(NT, NT == 256 ? 3 : 1) sample_compact_reg_kernel(SampleArgs a) {
+__global__ void __launch_bounds__(NT, NT == 256 ? 4 : 1) sample_compact_reg_kernel(SampleArgs a) {
     constexpr int NW = NT / 32;
     constexpr int PER = 4 * G;  // blocks per thread (<= 32: the masks are 32-bit)
     // the row is staged through shared memory with coalesced loads; thread
