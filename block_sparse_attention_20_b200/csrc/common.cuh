@@ -35,6 +35,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// 16-byte global -> shared copy that bypasses the registers (cp.async); with
+// keep == false nothing is read and the 16 bytes are zero-filled
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, bool keep) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
+                 "l"(__cvta_generic_to_global(src)), "r"(keep ? 16 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                  : "memory");
@@ -390,6 +400,17 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col_byte
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// 2^x of two values by one special-function-unit instruction: the pair is
+// rounded to fp16 (lo, hi), exponentiated in fp16 and widened back to fp32.
+// Inputs below -25 give +0, -inf gives +0.
+__device__ __forceinline__ float2 ex2_pair_f16(float2 x) {
+    uint32_t h, y;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(h));
+    const __half2 e = *reinterpret_cast<const __half2 *>(&y);
+    return __half22float2(e);
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -7,7 +7,8 @@
 // in shared memory as bf16 (exact copies of the inputs).  Per round:
 //   - distances: ||c_j||^2 - 2 q.c_j, the dot products on the tensor cores
 //     (mma.sync m16n8k16, bf16 in, fp32 accumulate; fragments by ldmatrix,
-//     the centroids' shared by a warp's two 16-row tiles) with each fp32 centroid
+//     the centroids' shared by a warp's two 16-row tiles; eight independent
+//     accumulation chains) with each fp32 centroid
 //     split into a bf16 high part and a bf16 residual, so the products carry
 //     about 16 significant bits of the centroid; warp w takes rows
 //     32w..32w+31; the argmin (ties to the lower index) is reduced across the
@@ -15,9 +16,11 @@
 //   - update: cluster sizes from warp ballots (each warp counts its own 32
 //     rows right after assigning them); the per-cluster sums of the
 //     rows are one more tensor-core product, onehot(assignment)^T . Q
-//     (16 x 128 times 128 x D, exact products, fp32 accumulation in the
-//     hardware's fixed order, so the result is deterministic); centroid =
-//     sum * (1/size), written with its bf16 operand parts.
+//     (16 x 128 times 128 x D, exact products, fp32 accumulation in a fixed
+//     order, so the result is deterministic); centroid = sum * (1/size),
+//     written with its bf16 operand parts, and each warp leaves the squared
+//     norm of its quarter of the dimensions for the next assignment (two
+//     block-wide barriers per round).
 //
 // Rules (open in the abstract, fixed here): C_eff = min(C, n) clusters;
 // centroid j starts at row floor(j*n/C_eff); squared Euclidean distance,
@@ -67,7 +70,7 @@ __device__ __forceinline__ uint32_t onehot_pair(bool lo, bool hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a) {
+__global__ void __launch_bounds__(kKmThreads, 5) kmeans_qblock_kernel(KmeansArgs a) {
     constexpr int LDQ = D + 8;  // bf16 row stride: 4*row + column-pair spreads the banks
     const int C = a.C;
     const int CP = C <= 8 ? 8 : 16;  // centroid rows held (one or two 8-wide MMA tiles)
@@ -76,7 +79,7 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
     float *cent = reinterpret_cast<float *>(km_smem + 128 * LDQ * 2);            // [CP][D]
     __nv_bfloat16 *chi = reinterpret_cast<__nv_bfloat16 *>(cent + CP * D);       // [CP][LDQ]
     __nv_bfloat16 *clo = chi + CP * LDQ;                                         // [CP][LDQ]
-    __shared__ float cnorm[kMaxC];
+    __shared__ float cnp_s[4][kMaxC];  // squared centroid norms, partial per warp (dimension quarter)
     __shared__ int assign_s[128];
     __shared__ int wcnt_s[4][kMaxC];
 
@@ -91,16 +94,18 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
         const __nv_bfloat16 *qblk = a.Q + a.st.head_base(bh) + (int64_t)i * 128 * a.st.sT;
 
         // the block's queries (each row's 16-byte chunks coalesced; rows sT
-        // apart); missing rows are zero
+        // apart), copied straight into shared memory so all of a thread's
+        // copies are in flight at once; missing rows are zero-filled
         {
             constexpr int CPR = D / 8;  // 16-byte chunks per row
-#pragma unroll 4
+#pragma unroll
             for (int c = tid; c < 128 * CPR; c += kKmThreads) {
                 const int r = c / CPR, x8 = c % CPR;
-                *reinterpret_cast<uint4 *>(qs + r * LDQ + x8 * 8) =
-                    r < n ? __ldg(reinterpret_cast<const uint4 *>(qblk + (int64_t)r * a.st.sT) + x8)
-                          : make_uint4(0, 0, 0, 0);
+                cp_async16_zfill(qs + r * LDQ + x8 * 8,
+                                 reinterpret_cast<const uint4 *>(qblk + (int64_t)(r < n ? r : 0) * a.st.sT) + x8,
+                                 r < n);
             }
+            cp_async_wait_all();
         }
         __syncthreads();
         // a centroid coordinate and its tensor-core operands: bf16 high part and
@@ -116,21 +121,23 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
             put(j, x, j < ce ? __bfloat162float(qs[(j * n) / ce * LDQ + x]) : 0.0f);
         }
         __syncthreads();
+        // squared norms of the seeds (warp w takes centroids w, w+4, ...; lanes
+        // split the dimensions); later rounds get them from the update
+        for (int j = warp; j < CP; j += 4) {
+            float s2 = 0.0f;
+#pragma unroll
+            for (int x = lane; x < D; x += 32) s2 = fmaf(cent[j * D + x], cent[j * D + x], s2);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+            if (lane == 0) {
+                cnp_s[0][j] = s2;
+                cnp_s[1][j] = cnp_s[2][j] = cnp_s[3][j] = 0.0f;
+            }
+        }
+        __syncthreads();
 
         const int rounds = a.iters > 0 ? a.iters : 1;
         for (int it = 0; it < rounds; ++it) {
-            // ---- squared norms of the centroids (operands were written with them) ----
-            // warp w takes centroids w, w+4, ...; lanes split the dimensions
-            for (int j = warp; j < CP; j += 4) {
-                float s = 0.0f;
-#pragma unroll
-                for (int x = lane; x < D; x += 32) s = fmaf(cent[j * D + x], cent[j * D + x], s);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                if (lane == 0) cnorm[j] = s;
-            }
-            __syncthreads();
-
             // ---- assignment: q.c on tensor cores, argmin over centroids ----
             // warp w: rows 32w..32w+31 as two 16-row MMA tiles; per 16-dim step one
             // ldmatrix of each query tile and one of the centroids' hi and lo parts
@@ -147,24 +154,37 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
             const __nv_bfloat16 *qa = qs + (warp * 32 + (lane & 15)) * LDQ + (lane >> 4) * 8;
             for (int t = 0; t < nt; ++t) {
                 const __nv_bfloat16 *cb = (lane < 16 ? chi : clo) + (t * 8 + (lane & 7)) * LDQ + ((lane >> 3) & 1) * 8;
-                float acc[2][4];
+                // eight independent accumulation chains: query tile m, centroid
+                // part (hi, lo) and the parity of the 16-dimension step
+                float acc[2][2][2][4];
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) acc[m][u] = 0.0f;
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int kp = 0; kp < 2; ++kp)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) acc[m][h][kp][u] = 0.0f;
 #pragma unroll
                 for (int k0 = 0; k0 < D; k0 += 16) {
+                    const int kp = (k0 >> 4) & 1;
                     uint32_t bf[4];  // hi (k0..7, k8..15), lo (k0..7, k8..15)
                     ldsm_x4(bf, cb + k0);
 #pragma unroll
                     for (int m = 0; m < 2; ++m) {
                         uint32_t af[4];
                         ldsm_x4(af, qa + m * 16 * LDQ + k0);
-                        mma_bf16_16816(acc[m], af, bf[0], bf[1]);
-                        mma_bf16_16816(acc[m], af, bf[2], bf[3]);
+                        mma_bf16_16816(acc[m][0][kp], af, bf[0], bf[1]);
+                        mma_bf16_16816(acc[m][1][kp], af, bf[2], bf[3]);
                     }
                 }
-                // acc[m][0..1]: row g, centroids t*8+2cq+{0,1}; acc[m][2..3]: row g+8
+                float cn[2];  // squared norms of this lane's two centroids
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int j = t * 8 + 2 * cq + u;
+                    cn[u] = (cnp_s[0][j] + cnp_s[1][j]) + (cnp_s[2][j] + cnp_s[3][j]);
+                }
+                // acc[m][.][.][0..1]: row g, centroids t*8+2cq+{0,1}; [2..3]: row g+8
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -172,8 +192,9 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int j = t * 8 + 2 * cq + u;
-                            const float dj = j < ce ? fmaf(-2.0f, acc[m][2 * h + u], cnorm[j])
-                                                    : __int_as_float(0x7f800000);
+                            const int e = 2 * h + u;
+                            const float dot = (acc[m][0][0][e] + acc[m][0][1][e]) + (acc[m][1][0][e] + acc[m][1][1][e]);
+                            const float dj = j < ce ? fmaf(-2.0f, dot, cn[u]) : __int_as_float(0x7f800000);
                             if (dj < bestd[m][h]) { bestd[m][h] = dj; besti[m][h] = j; }
                         }
             }
@@ -215,14 +236,17 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
             // takes the column tiles of dimensions [w*D/4, (w+1)*D/4)
             {
                 constexpr int NT = D / 32;  // 8-wide column tiles per warp
-                float acc[NT][4];
+                float acc[2][NT][4];            // [parity of the 16-row step][column tile]
 #pragma unroll
-                for (int t = 0; t < NT; ++t)
+                for (int kp = 0; kp < 2; ++kp)
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) acc[t][u] = 0.0f;
+                    for (int t = 0; t < NT; ++t)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) acc[kp][t][u] = 0.0f;
                 const int n0w = warp * NT * 8;
-#pragma unroll 2
+#pragma unroll
                 for (int k0 = 0; k0 < 128; k0 += 16) {
+                    const int kp = (k0 >> 4) & 1;
                     const int q0 = assign_s[k0 + 2 * cq], q1 = assign_s[k0 + 2 * cq + 1];
                     const int q8 = assign_s[k0 + 2 * cq + 8], q9 = assign_s[k0 + 2 * cq + 9];
                     uint32_t af[4];
@@ -238,24 +262,36 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_qblock_kernel(KmeansArgs a)
                             qs + (k0 + (mi & 1) * 8 + (lane & 7)) * LDQ + n0w + (t + (mi >> 1)) * 8;
                         uint32_t b[4];
                         ldsm_x4_trans(b, ra);
-                        mma_bf16_16816(acc[t], af, b[0], b[1]);
-                        mma_bf16_16816(acc[t + 1], af, b[2], b[3]);
+                        mma_bf16_16816(acc[kp][t], af, b[0], b[1]);
+                        mma_bf16_16816(acc[kp][t + 1], af, b[2], b[3]);
                     }
                 }
-                // acc[t]: [0..1] cluster g, dimensions n0w+8t+2cq+{0,1}; [2..3] cluster g+8
+                // acc[.][t]: [0..1] cluster g, dimensions n0w+8t+2cq+{0,1}; [2..3] cluster g+8.
+                // Each updated centroid also leaves the squared norm of this warp's
+                // D/4 dimensions of it for the next assignment (the four lanes of a
+                // quad hold one cluster's values)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int j = g + 8 * h;
-                    if (j >= ce) continue;
-                    const int c = wcnt_s[0][j] + wcnt_s[1][j] + wcnt_s[2][j] + wcnt_s[3][j];
-                    if (c == 0) continue;  // an empty cluster keeps its centroid
-                    const float inv = __frcp_rn((float)c);  // sum / size as sum * (1/size)
+                    const int c = j < ce ? wcnt_s[0][j] + wcnt_s[1][j] + wcnt_s[2][j] + wcnt_s[3][j] : 0;
+                    // c == 0: an empty cluster keeps its centroid (and its norm)
+                    const float inv = c > 0 ? __frcp_rn((float)c) : 0.0f;  // sum / size as sum * (1/size)
+                    float pn = 0.0f;
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
                         const int x = n0w + 8 * t + 2 * cq;
-                        put(j, x, __fmul_rn(acc[t][2 * h], inv));
-                        put(j, x + 1, __fmul_rn(acc[t][2 * h + 1], inv));
+                        const float c0 = __fmul_rn(acc[0][t][2 * h] + acc[1][t][2 * h], inv);
+                        const float c1 = __fmul_rn(acc[0][t][2 * h + 1] + acc[1][t][2 * h + 1], inv);
+                        pn = fmaf(c0, c0, pn);
+                        pn = fmaf(c1, c1, pn);
+                        if (c > 0) {
+                            put(j, x, c0);
+                            put(j, x + 1, c1);
+                        }
                     }
+                    pn += __shfl_xor_sync(0xffffffffu, pn, 1);
+                    pn += __shfl_xor_sync(0xffffffffu, pn, 2);
+                    if (c > 0 && cq == 0) cnp_s[warp][j] = pn;
                 }
             }
             __syncthreads();
