@@ -60,12 +60,6 @@ constexpr float kRescaleThreshold = 8.0f;
 #define ABATT_ATTN_POLY_OF_8 0
 #endif
 constexpr int kAttnPolyOf8 = ABATT_ATTN_POLY_OF_8;
-// 1: the softmax exponentials go through the fp16 pair form of ex2 (two per
-// special-function-unit instruction); 0: one fp32 ex2 per value
-#ifndef ABATT_ATTN_EX2_F16
-#define ABATT_ATTN_EX2_F16 0
-#endif
-constexpr bool kAttnEx2F16 = ABATT_ATTN_EX2_F16 != 0;
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -623,8 +617,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         float2 p;
                         if (((c * 16 + (j >> 1)) & 7) < kAttnPolyOf8) {
                             p = exp2_poly2<3>(x);
-                        } else if (kAttnEx2F16) {
-                            p = ex2_pair_f16(x);
                         } else {
                             p.x = ex2_approx(x.x);
                             p.y = ex2_approx(x.y);

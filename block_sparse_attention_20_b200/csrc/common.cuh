@@ -402,17 +402,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// 2^x of two values by one special-function-unit instruction: the pair is
-// rounded to fp16 (lo, hi), exponentiated in fp16 and widened back to fp32.
-// Inputs below -25 give +0, -inf gives +0.
-__device__ __forceinline__ float2 ex2_pair_f16(float2 x) {
-    uint32_t h, y;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x.y), "f"(x.x));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(h));
-    const __half2 e = *reinterpret_cast<const __half2 *>(&y);
-    return __half22float2(e);
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
