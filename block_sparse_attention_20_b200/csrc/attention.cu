@@ -579,19 +579,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             if (k == tail_k && col % BK >= tail_keep) v[c][j] = __float_as_uint(kNegInf);
                         }
                 }
-                float bmax[HB];
+                // raw maximum of each block's columns in this half (a tree: short
+                // dependency chains), then the half's maximum of scaled + weighted
+                constexpr int VPB = 64 / HB;  // columns of one block (part) in this half
+                float hm[HB];
 #pragma unroll
-                for (int k = 0; k < HB; ++k) bmax[k] = kNegInf;
+                for (int k = 0; k < HB; ++k) {
+                    float w[VPB];
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const int k = BPT >= 2 ? (c * 32 + j) / BK : 0;
-                        bmax[k] = fmax3f(bmax[k], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
+                    for (int e = 0; e < VPB; ++e) {
+                        const int col = k * VPB + e;  // 0..63 within the half
+                        w[e] = __uint_as_float(v[col >> 5][col & 31]);
                     }
-                float hmax = kNegInf;
-#pragma unroll
-                for (int k = 0; k < HB; ++k) hmax = fmaxf(hmax, fmaf(bmax[k], a.scale_log2, bias[k]));
+                    hm[k] = fmaf(max_tree<VPB>(w), a.scale_log2, bias[k]);
+                }
+                const float hmax = max_tree<HB>(hm);
                 const float tmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, 16));
                 const bool need = tmax > m_run + kRescaleThreshold;
                 const float m_use = need ? tmax : m_run;

@@ -358,6 +358,30 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
     return r;
 }
 
+// Maximum of N values as a tree of 3-input maxima (depth ceil(log3 N)
+// instead of a chain of N/2): exact, so any order gives the same result.
+template <int N>
+__device__ __forceinline__ float max_tree(const float *w) {
+    if constexpr (N == 1) {
+        return w[0];
+    } else if constexpr (N == 2) {
+        return fmaxf(w[0], w[1]);
+    } else if constexpr (N == 3) {
+        return fmax3f(w[0], w[1], w[2]);
+    } else {
+        constexpr int M = (N + 2) / 3;
+        float u[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const int b = 3 * i;
+            if (b + 2 < N) u[i] = fmax3f(w[b], w[b + 1], w[b + 2]);
+            else if (b + 1 < N) u[i] = fmaxf(w[b], w[b + 1]);
+            else u[i] = w[b];
+        }
+        return max_tree<M>(u);
+    }
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major = false) {
     return (1u << 4)                         // D format: f32
            | (1u << 7)                       // A format: bf16
